@@ -1,0 +1,84 @@
+/*
+ * nvfp4_oracle.h -- plain CPU reference of the grouped row-scaled NVFP4 cast.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may include, link or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline use it. It shares no code with the CUDA library.
+ *
+ * Sources (web pages the method is taken from):
+ *  - TransformerEngine #3649, "single-launch grouped row-scaled NVFP4 cast",
+ *    Description: a grouped amax over the packed (sum_M, K) buffer yields
+ *    rowwise [sum_M] and columnwise [num_tensors*K] amax in one pass; a
+ *    grouped cast consumes both and writes packed FP4 data and scales.
+ *  - TransformerEngine #2931, "Implement per-token NVFP4 fprop recipe",
+ *    Changes and sequence diagram: per-token (row) amax as the FP32
+ *    second-level scale, FP8 (E4M3) block scales, FP4 data; dequantize looks
+ *    up the amax of the element's row; the GEMM runs with amax = 1 and its
+ *    rows are multiplied back by the row amax.
+ *  - TransformerEngine #3324, "Enable NVFP4 row-scaled (per-token) backward
+ *    for GroupedLinear", summary: per-column amax for the columnwise operand.
+ *  - TransformerEngine #3824, "What this changes", item 2: a 0-element split
+ *    must not fail.
+ *
+ * All floating point is IEEE-754 binary32, round to nearest even, one
+ * rounding per written operation (the translation unit is compiled with
+ * -ffp-contract=off on SSE). Return values: 0 = ok, nonzero = error (see
+ * NVO_E_* below).
+ */
+#ifndef NVFP4_ORACLE_H
+#define NVFP4_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NVO_OK 0
+#define NVO_E_ARG 1        /* bad size, split or pointer */
+#define NVO_E_NONFINITE 2  /* an input element is Inf or NaN */
+
+/* format helpers */
+float nvo_bf16_to_f32(uint16_t bits);
+float nvo_e2m1_decode(uint8_t code);          /* low 4 bits used */
+uint8_t nvo_e2m1_encode(float y);             /* RNE onto E2M1, saturating */
+float nvo_e4m3_decode(uint8_t code);          /* E4M3 "FN": NaN for 0x7F/0xFF */
+uint8_t nvo_e4m3_encode(float v);             /* RNE onto E4M3, saturating */
+
+/* element-wise array forms of the two encoders (test helpers) */
+void nvo_e2m1_encode_array(const float* y, int64_t n, uint8_t* out);
+void nvo_e4m3_encode_array(const float* v, int64_t n, uint8_t* out);
+
+/* second-level scales of one amax value a */
+float nvo_s_enc(float a);
+float nvo_s_dec(float a);
+
+/* one 16-element block: block scale byte and 16 codes (one per element) */
+void nvo_block_encode(const float* x16, float s_enc, uint8_t* s8, uint8_t* codes16);
+
+/* grouped amax (both directions). row_amax [sum_M], col_amax [E*K];
+ * either output may be NULL to skip that direction. */
+int nvo_group_amax(const uint16_t* x, int64_t sum_M, int64_t K,
+                   const int64_t* m_splits, int32_t E,
+                   float* row_amax, float* col_amax);
+
+/* grouped cast. Rowwise outputs: row_data [sum_M, K/2], row_scale
+ * [sum_M, K/16], row_s2 [sum_M]. Colwise outputs: per group g a transposed
+ * slice, col_data at byte K*o_g/2 of shape [K, m_g/2], col_scale at byte
+ * K*o_g/16 of shape [K, m_g/16], col_s2 [E*K]. A direction whose three
+ * pointers are NULL is skipped. */
+int nvo_group_cast(const uint16_t* x, int64_t sum_M, int64_t K,
+                   const int64_t* m_splits, int32_t E,
+                   const float* row_amax, const float* col_amax,
+                   uint8_t* row_data, uint8_t* row_scale, float* row_s2,
+                   uint8_t* col_data, uint8_t* col_scale, float* col_s2);
+
+/* dequantize one row-major quantized matrix [rows, cols] with one s2 per row */
+int nvo_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
+                   int64_t rows, int64_t cols, float* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif
