@@ -1,0 +1,401 @@
+"""Benchmark of the grouped row-scaled NVFP4 cast (grouped amax + grouped cast).
+
+One step = one pass of the whole hot path over one batch: nvfp4_group_amax
+(row and per-group column amax, one read of x) then nvfp4_group_cast (rowwise
+and colwise FP4 codes, E4M3 block scales, FP32 decode scales). The default
+workload is the DeepSeek-V3-shaped MoE input: K = 7168, 256 experts, 8192
+tokens x top-8 = 65536 routed rows, Zipf(1.1) expert popularity, ~10% empty
+experts, every group zero-padded to a multiple of 128 rows (synthetic, seeded).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+casts its own copy of the workload (expert parallelism: each GPU casts its
+local experts; no collective on the data path) and rank 0 prints one JSON line.
+
+Metric: input Gelem/s (sum_M*K elements per step). Reported beside it: HBM
+GB/s of the method's algorithmic bytes and the roofline of the dominant
+kernel against the measured HBM copy bandwidth of this machine's B200s.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "grouped NVFP4 cast: input Gelem/s and HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------- bytes
+
+def algorithmic_bytes(sum_M: int, K: int, E: int):
+    """Bytes each step must move, by kernel (two reads of x: one per step of
+    the method; outputs written once)."""
+    N = sum_M * K
+    amax = 2 * N + 4 * sum_M + 4 * E * K                     # read x; write row/col amax
+    cast = (2 * N                                             # read x
+            + 4 * sum_M + 4 * E * K                           # read row/col amax
+            + N // 2 + N // 16 + 4 * sum_M                    # rowwise codes, scales, S_dec
+            + N // 2 + N // 16 + 4 * E * K)                   # colwise codes, scales, S_dec
+    return {"amax": amax, "cast": cast, "step": amax + cast}
+
+
+def output_bytes(sum_M: int, K: int, E: int) -> int:
+    N = sum_M * K
+    return 2 * (N // 2 + N // 16) + 4 * sum_M + 4 * E * K
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    d = os.path.join(ROOT, "nvfp4_row_scaled_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only if it was
+    taken on the current kernel sources and the same workload."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    r = rec.get(kernel)
+    if not r or r.get("source_hash") != kernel_source_hash() or r.get("workload") != workload:
+        return None
+    return r.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_sample(w, target_s: float = 12.0, max_threads: int = 64):
+    """Time the oracle (amax + cast, both directions) on a bounded sample of
+    the workload: whole groups, taken in order until the sample has about
+    target_s of CPU work, run one group per thread across the host cores."""
+    import numpy as np  # noqa: F401
+
+    import oracle
+    from nvfp4_row_scaled_b200 import workloads
+
+    xb = workloads.bits(w.x)
+    offs = workloads.row_offsets(w.m_splits)
+    groups = [(offs[g], m) for g, m in enumerate(w.m_splits) if m > 0]
+    cores = min(os.cpu_count() or 1, max_threads)
+
+    def one(o_m):
+        o, m = o_m
+        sub = xb[o:o + m]
+        ra, ca = oracle.group_amax(sub, [m])
+        oracle.group_cast(sub, [m], ra, ca)
+        return m * w.K
+
+    # calibrate on one small group
+    small = min(groups, key=lambda g: g[1])
+    t0 = time.perf_counter()
+    one(small)
+    rate = small[1] * w.K / max(time.perf_counter() - t0, 1e-6)  # elements/s per thread
+    budget = rate * target_s * cores
+    sample, n = [], 0
+    for gm in sorted(groups, key=lambda g: g[1]):
+        if n + gm[1] * w.K > budget and sample:
+            break
+        sample.append(gm)
+        n += gm[1] * w.K
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        done = sum(ex.map(one, sample))
+    dt = time.perf_counter() - t0
+    return {"value": done / dt / 1e9, "unit": "Gelem/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample)} whole groups ({sum(m for _, m in sample)} rows x {w.K}, "
+                      f"{done / 1e6:.1f} M elements) of the workload, amax + cast both directions, "
+                      f"one group per thread, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------- the bench
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--tokens", type=int, default=8192, help="scales the workload (tests only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    from nvfp4_row_scaled_b200 import abi, workloads
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    w = workloads.config3(tokens=args.tokens)
+    K, E, M = w.K, w.E, w.sum_M
+    N = M * K
+    splits = w.m_splits
+    x_host = w.x.pin_memory()
+    x = x_host.to(dev)
+    ra, ca = abi.alloc_amax(M, K, E, dev)
+    out = abi.alloc_outputs(M, K, E, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        abi.nvfp4_group_amax(x, splits, ra, ca)
+        abi.nvfp4_group_cast(x, splits, ra, ca, out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # ---- device-timed region: K steps, per-kernel events on the launch stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        abi.nvfp4_group_amax(x, splits, ra, ca)
+        ev[i][1].record(stream)
+        abi.nvfp4_group_cast(x, splits, ra, ca, out)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    amax_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    cast_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+
+    # ---- end to end through the C ABI with host buffers (pinned)
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+    e2e_steps = max(3, min(args.steps, 5))
+    step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        for k, v in out.items():
+            host_out[k].copy_(v, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * N / (ms_per_step * 1e-3) / 1e9
+    b = algorithmic_bytes(M, K, E)
+    peak, peak_kind = hbm_peak()
+    dominant = "cast" if cast_ms >= amax_ms else "amax"
+    dom_ms = cast_ms if dominant == "cast" else amax_ms
+    achieved = b[dominant] / (dom_ms * 1e-3) / 1e9
+    workload_name = w.name
+    traffic = traffic_record("group_cast_kernel" if dominant == "cast" else "group_amax_kernel",
+                             workload_name)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(w)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "Gelem/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; no dataset)",
+        "config": {
+            "workload": workload_name,
+            "K": K, "experts": E, "sum_M": M, "routed_rows": 8 * args.tokens,
+            "elements_per_step": N,
+            "path": "host-split nvfp4_group_amax + nvfp4_group_cast, rowwise + colwise",
+            "l2": f"inputs larger than L2 ({2 * N / 1e9:.2f} GB bf16 > 126 MB); no flush",
+            "parallelism": f"ep{world} (each GPU casts its own experts)",
+        },
+        "hbm_gbs": round(b["step"] / (ms_per_step * 1e-3) / 1e9, 1),
+        "hbm_frac_of_peak": round(b["step"] / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        "kernels_ms": {"amax": round(amax_ms, 4), "cast": round(cast_ms, 4)},
+        "roofline": {
+            "kernel": f"group_{dominant}_kernel",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": b[dominant],
+        },
+        "cpu_baseline": cpu,
+        "e2e": {
+            "value": round(world * N / (e2e_ms * 1e-3) / 1e9, 3),
+            "unit": "Gelem/s",
+            "h2d_bytes_per_step": 2 * N,
+            "d2h_bytes_per_step": output_bytes(M, K, E),
+        },
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def reference_arm(args, rank: int, world: int):
+    """The oracle as the reference arm: each step is the oracle's amax + cast
+    on a bounded sample of the same workload, on the host cores."""
+    if rank != 0:
+        return
+    from nvfp4_row_scaled_b200 import workloads
+    w = workloads.config3(tokens=args.tokens)
+    per_step = max(2.0, 60.0 / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, target_s=per_step / 4)
+    vals, info = [], None
+    for _ in range(args.steps):
+        info = cpu_oracle_sample(w, target_s=per_step)
+        vals.append(info["value"])
+    value = statistics.median(vals)
+    N = w.sum_M * w.K
+    line = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 4), "unit": "Gelem/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(N / (value * 1e9) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 (oracle arithmetic on bf16 input)",
+        "data": "synthetic (seeded; no dataset)",
+        "config": {"workload": w.name, "K": w.K, "experts": w.E, "sum_M": w.sum_M,
+                   "note": "each step times the oracle on a bounded sample of the workload"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "Gelem/s", "cores": info["cores"],
+                         "kind": "oracle", "sample": info["sample"]},
+        "e2e": {"value": round(value, 4), "unit": "Gelem/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

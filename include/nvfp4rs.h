@@ -1,0 +1,200 @@
+/*
+ * nvfp4rs.h -- C ABI of the grouped row-scaled (per-token) NVFP4 cast for
+ * NVIDIA B200 (sm_100a). Library: libnvfp4rs.so.
+ *
+ * The method (web pages it follows):
+ *  - TransformerEngine #3649, "single-launch grouped row-scaled NVFP4 cast",
+ *    Description: the cast of packed MoE expert activations runs as two
+ *    single-launch kernels -- a grouped amax over the packed (sum_M, K) buffer
+ *    that yields rowwise [sum_M] and columnwise [num_tensors*K] amax in one
+ *    pass, then a grouped cast that consumes both -- and each step has a
+ *    graph-safe counterpart that reads the routing from device
+ *    first_dims / tensor_offsets instead of host splits, sharing the device
+ *    body so that the outputs are byte-identical.
+ *  - TransformerEngine #2931, "Implement per-token NVFP4 fprop recipe",
+ *    Changes and Important Files Changed: per-token (row) amax as the FP32
+ *    second-level scale of NVFP4 (E2M1 data, E4M3 block scales), and a
+ *    dequantize that looks up the amax of each element's row.
+ *  - TransformerEngine #3324, "Enable NVFP4 row-scaled (per-token) backward
+ *    for GroupedLinear", summary: per-column amax for the columnwise
+ *    (transposed) operand.
+ *
+ * Numerics (identical, byte for byte, to the CPU oracle of this project):
+ *   S_enc(a) = a == 0 ? 1 : min(fl(2688 / a), FLT_MAX)      2688 = 6 * 448
+ *   S_dec(a) = fl(a / 2688)
+ *   per 16-element block: s8  = E4M3_rne_satfinite(fl(fl(bmax / 6) * S_enc))
+ *                         enc = s8 == 0 ? 0 : min(fl(S_enc / e4m3(s8)), FLT_MAX)
+ *                         code_j = E2M1_rne_satfinite(fl(x_j * enc)), sign kept
+ *   dequantize: x_hat = fl((e2m1(code) * e4m3(s8)) * S_dec)
+ * All float arithmetic is IEEE binary32, round to nearest even, no FMA.
+ *
+ * Layouts (all row-major, all compact):
+ *   x          bf16  [rows, K]
+ *   row_amax   fp32  [rows]
+ *   col_amax   fp32  [E * K]           group g, column k at g*K + k
+ *   row_data   u8    [rows, K/2]       element 2j in the low nibble of byte j
+ *   row_scale  u8    [rows, K/16]      one E4M3 byte per 16-element block
+ *   row_s2     fp32  [rows]            S_dec of the row amax
+ *   col_data   u8    group g at byte offset K*o_g/2, shape [K, m_g/2]
+ *                    (the group's transpose; element = row within the group)
+ *   col_scale  u8    group g at byte offset K*o_g/16, shape [K, m_g/16]
+ *   col_s2     fp32  [E * K]           S_dec of the column amax
+ * where o_g = m_0 + ... + m_{g-1} is the first row of group g.
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller allocates and owns every buffer (device memory
+ *    unless stated). The library allocates nothing, never synchronises the
+ *    stream and never reads device memory from the host. Every call only
+ *    enqueues work (memsets and kernels) on `stream`.
+ *  - Errors: argument errors are found on the host before anything is
+ *    enqueued and returned synchronously; nothing is written then. A failed
+ *    CUDA launch returns NVFP4_ERR_CUDA. The graph-safe calls check the device
+ *    routing on the device: a violation is written to *status_dev and the
+ *    kernels write no output; they never trap and never hang.
+ *  - Fast-path requirements (else NVFP4_ERR_UNSUPPORTED): K % 128 == 0,
+ *    every group size m_g % 128 == 0 (the 128-row alignment of the grouped
+ *    GEMM's scale layout), num_groups <= NVFP4_MAX_GROUPS, rows < 2^31, and
+ *    every pointer 16-byte aligned. Inputs must be finite (a non-finite input
+ *    gives unspecified codes, never a fault).
+ *  - Empty groups (m_g == 0) are allowed: their col_amax and col_s2 are 0
+ *    and they own no bytes of col_data / col_scale.
+ */
+#ifndef NVFP4RS_H
+#define NVFP4RS_H
+
+#include <stdint.h>
+
+#include <cuda_runtime_api.h> /* cudaStream_t */
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* null pointer, negative size, splits that do not add up, K % 16 */
+  NVFP4_ERR_UNSUPPORTED = 2, /* valid, but outside the fast path (see above) */
+  NVFP4_ERR_CUDA = 3,        /* a CUDA call or launch failed */
+  NVFP4_ERR_ROUTING = 4      /* graph-safe only: device routing is inconsistent */
+} nvfp4_status;
+
+#define NVFP4_MAX_GROUPS 1024
+
+/* every entry point is exported; everything else in the library is hidden */
+#if defined(__GNUC__)
+#define NVFP4RS_API __attribute__((visibility("default")))
+#else
+#define NVFP4RS_API
+#endif
+
+/* Output buffers of the grouped cast (device pointers). A direction whose
+ * three pointers are all NULL is skipped; a direction with some but not all
+ * three set is NVFP4_ERR_INVALID_ARG. */
+typedef struct {
+  uint8_t* row_data;  /* [rows, K/2]   */
+  uint8_t* row_scale; /* [rows, K/16]  */
+  float* row_s2;      /* [rows]        */
+  uint8_t* col_data;  /* per group [K, m_g/2] at byte K*o_g/2   */
+  uint8_t* col_scale; /* per group [K, m_g/16] at byte K*o_g/16 */
+  float* col_s2;      /* [E*K]         */
+} nvfp4_outputs;
+
+/*
+ * Grouped amax, host-split routing (TransformerEngine #3649, Description:
+ * one launch reads the packed bf16 buffer once and yields both the per-row
+ * amax and the per-group per-column amax; the per-column amax is the
+ * columnwise operand's scale source, as in #3324).
+ *   x_bf16         device, bf16 [sum_M, K], read once
+ *   sum_M, K       rows and columns; sum_M == sum of m_splits_host
+ *   m_splits_host  HOST array [num_groups] of rows per group; read during the
+ *                  call only (copied into kernel parameters)
+ *   row_amax       device fp32 [sum_M], or NULL to skip rows
+ *   col_amax       device fp32 [num_groups*K], or NULL to skip columns; it is
+ *                  zeroed on `stream` by this call first
+ * One launch (plus one memset of col_amax).
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
+                              const int64_t* m_splits_host, int32_t num_groups,
+                              float* row_amax, float* col_amax, cudaStream_t stream);
+
+/*
+ * Grouped cast, host-split routing (TransformerEngine #3649, Description:
+ * the second launch, which takes both amax vectors as its scale sources;
+ * #2931, Changes: per-token NVFP4 quantization). Writes, from one read of each tile of x, the rowwise blocks
+ * (16 along K, scaled by the row's amax) and the colwise blocks (16 along the
+ * rows of a group, scaled by the group's column amax), plus the FP32 decode
+ * scales row_s2 / col_s2.
+ *   row_amax, col_amax  device, as written by nvfp4_group_amax (row_amax is
+ *                       needed if the row direction is requested, col_amax
+ *                       if the column direction is)
+ *   out                 HOST pointer to the output descriptor (device buffers)
+ * One launch.
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
+                              const int64_t* m_splits_host, int32_t num_groups,
+                              const float* row_amax, const float* col_amax,
+                              const nvfp4_outputs* out, cudaStream_t stream);
+
+/*
+ * Grouped amax, graph-safe routing (TransformerEngine #3649, Description:
+ * the twin of the host-split call whose group boundaries come from device
+ * arrays, first_dims and tensor_offsets, rather than from host splits). Nothing about
+ * the routing is read on the host, so the call can be captured in a CUDA
+ * graph once and replayed after the routing buffers change on the device.
+ * The device body is the one nvfp4_group_amax runs, so for equal routing
+ * the outputs are byte-identical.
+ *   capacity_rows       rows allocated in x (the grid is sized by it); rows at
+ *                       or beyond the routed total are neither read nor written
+ *   first_dims_dev      device int64 [num_groups]: rows of each group
+ *   tensor_offsets_dev  device int64 [num_groups+1]: ELEMENT offset of each
+ *                       group (row offset * K); [0] == 0, and
+ *                       first_dims[g]*K == offsets[g+1] - offsets[g];
+ *                       offsets[num_groups] / K <= capacity_rows
+ *   status_dev          device int32 [1]: set to 0 by this call, then to
+ *                       NVFP4_ERR_ROUTING (inconsistent routing) or
+ *                       NVFP4_ERR_UNSUPPORTED (a group not a multiple of 128
+ *                       rows) by the kernel, which then writes no amax
+ * One launch plus memsets of status and col_amax.
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                        const int64_t* first_dims_dev,
+                                        const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                        float* row_amax, float* col_amax, int32_t* status_dev,
+                                        cudaStream_t stream);
+
+/*
+ * Grouped cast, graph-safe routing: nvfp4_group_cast with the routing of
+ * nvfp4_group_amax_graphsafe (same arguments, same status rules; status_dev
+ * is reset to 0 by this call too). Byte-identical to nvfp4_group_cast for
+ * equal routing. One launch plus one memset of status.
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                        const int64_t* first_dims_dev,
+                                        const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                        const float* row_amax, const float* col_amax,
+                                        const nvfp4_outputs* out, int32_t* status_dev,
+                                        cudaStream_t stream);
+
+/*
+ * Dequantize one quantized matrix [rows, cols] to FP32 with one decode scale
+ * per row (TransformerEngine #2931, Important Files Changed: the dequantize
+ * kernel looks up the amax of the element's row, tensor_amax[y]).
+ *   data   device u8 [rows, cols/2], scale device u8 [rows, cols/16],
+ *   s2     device fp32 [rows], out device fp32 [rows, cols]
+ * Rowwise output: pass row_data/row_scale/row_s2 with rows = sum_M, cols = K.
+ * Colwise output of group g: pass its slices with rows = K, cols = m_g and
+ * s2 = col_s2 + g*K. Requires cols % 16 == 0 (else NVFP4_ERR_INVALID_ARG),
+ * an 8-byte aligned data pointer and a 16-byte aligned out pointer (else
+ * NVFP4_ERR_UNSUPPORTED). One launch.
+ */
+NVFP4RS_API nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
+                              int64_t rows, int64_t cols, float* out_f32, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+NVFP4RS_API const char* nvfp4_status_string(nvfp4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4RS_H */

@@ -1,0 +1,204 @@
+"""Thin ctypes binding of ``libnvfp4rs.so`` (declared in ``include/nvfp4rs.h``).
+
+Argument marshalling only: every function here checks that tensors are CUDA,
+contiguous and of the right dtype, turns them into device pointers, passes the
+current torch stream, and raises ``NVFP4Error`` on a non-OK status. All of the
+method's work happens in the library's kernels. If the library is not built,
+every call raises; there is no fallback.
+
+Names follow the C entry points. Tensors:
+  x            bf16 [rows, K]
+  row_amax     fp32 [rows]          col_amax  fp32 [E*K]
+  row_data     uint8 [rows, K/2]    row_scale uint8 [rows, K/16]   row_s2 fp32 [rows]
+  col_data     uint8 [rows*K/2]     col_scale uint8 [rows*K/16]    col_s2 fp32 [E*K]
+(colwise buffers hold each group's transposed [K, m_g/2] / [K, m_g/16] slice
+at byte offsets K*o_g/2 and K*o_g/16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4rs.so")
+
+NVFP4_OK = 0
+NVFP4_ERR_INVALID_ARG = 1
+NVFP4_ERR_UNSUPPORTED = 2
+NVFP4_ERR_CUDA = 3
+NVFP4_ERR_ROUTING = 4
+NVFP4_MAX_GROUPS = 1024
+
+_lib = None
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {status_name(status)} ({status})")
+        self.status = status
+
+
+class Outputs(ctypes.Structure):
+    """Mirror of ``nvfp4_outputs``."""
+    _fields_ = [("row_data", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
+                ("row_s2", ctypes.c_void_p), ("col_data", ctypes.c_void_p),
+                ("col_scale", ctypes.c_void_p), ("col_s2", ctypes.c_void_p)]
+
+
+def lib():
+    """Open the library (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               f"`python -m nvfp4_row_scaled_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        L.nvfp4_group_amax.argtypes = [vp, i64, i64, vp, i32, vp, vp, vp]
+        L.nvfp4_group_cast.argtypes = [vp, i64, i64, vp, i32, vp, vp, ctypes.POINTER(Outputs), vp]
+        L.nvfp4_group_amax_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp, vp, vp]
+        L.nvfp4_group_cast_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp,
+                                                 ctypes.POINTER(Outputs), vp, vp]
+        L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, vp]
+        for f in ("nvfp4_group_amax", "nvfp4_group_cast", "nvfp4_group_amax_graphsafe",
+                  "nvfp4_group_cast_graphsafe", "nvfp4_dequantize"):
+            getattr(L, f).restype = ctypes.c_int
+        L.nvfp4_status_string.argtypes = [ctypes.c_int]
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_name(status: int) -> str:
+    return lib().nvfp4_status_string(int(status)).decode()
+
+
+# ----------------------------------------------------------- marshalling
+
+def _dev(t: Optional[torch.Tensor], dtype: torch.dtype, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _splits(m_splits: Sequence[int]):
+    arr = (ctypes.c_int64 * max(len(m_splits), 1))(*[int(m) for m in m_splits])
+    return arr, len(m_splits)
+
+
+def _outputs(out: Dict[str, torch.Tensor]) -> Outputs:
+    o = Outputs()
+    for name, dt in (("row_data", torch.uint8), ("row_scale", torch.uint8), ("row_s2", torch.float32),
+                     ("col_data", torch.uint8), ("col_scale", torch.uint8), ("col_s2", torch.float32)):
+        p = _dev(out.get(name), dt, name)
+        setattr(o, name, p.value if p is not None else None)
+    return o
+
+
+def _check(rc: int, what: str):
+    if rc != NVFP4_OK:
+        raise NVFP4Error(what, rc)
+
+
+# ------------------------------------------------------------ entry points
+
+def nvfp4_group_amax(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optional[torch.Tensor],
+                     col_amax: Optional[torch.Tensor], stream=None) -> None:
+    arr, E = _splits(m_splits)
+    rc = lib().nvfp4_group_amax(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
+                                _dev(row_amax, torch.float32, "row_amax"),
+                                _dev(col_amax, torch.float32, "col_amax"), _stream(stream))
+    _check(rc, "nvfp4_group_amax")
+
+
+def nvfp4_group_cast(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optional[torch.Tensor],
+                     col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
+                     stream=None) -> None:
+    arr, E = _splits(m_splits)
+    o = _outputs(out)
+    rc = lib().nvfp4_group_cast(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
+                                _dev(row_amax, torch.float32, "row_amax"),
+                                _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
+                                _stream(stream))
+    _check(rc, "nvfp4_group_cast")
+
+
+def nvfp4_group_amax_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
+                               tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
+                               col_amax: Optional[torch.Tensor], status: torch.Tensor,
+                               stream=None) -> None:
+    rc = lib().nvfp4_group_amax_graphsafe(
+        _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
+        _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
+        first_dims.numel(), _dev(row_amax, torch.float32, "row_amax"),
+        _dev(col_amax, torch.float32, "col_amax"), _dev(status, torch.int32, "status"),
+        _stream(stream))
+    _check(rc, "nvfp4_group_amax_graphsafe")
+
+
+def nvfp4_group_cast_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
+                               tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
+                               col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
+                               status: torch.Tensor, stream=None) -> None:
+    o = _outputs(out)
+    rc = lib().nvfp4_group_cast_graphsafe(
+        _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
+        _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
+        first_dims.numel(), _dev(row_amax, torch.float32, "row_amax"),
+        _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
+        _dev(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "nvfp4_group_cast_graphsafe")
+
+
+def nvfp4_dequantize(data: torch.Tensor, scale: torch.Tensor, s2: torch.Tensor, rows: int, cols: int,
+                     out: torch.Tensor, stream=None) -> None:
+    rc = lib().nvfp4_dequantize(_dev(data, torch.uint8, "data"), _dev(scale, torch.uint8, "scale"),
+                                _dev(s2, torch.float32, "s2"), int(rows), int(cols),
+                                _dev(out, torch.float32, "out"), _stream(stream))
+    _check(rc, "nvfp4_dequantize")
+
+
+# -------------------------------------------------------- buffer helpers
+
+def alloc_amax(rows: int, K: int, E: int, device="cuda"):
+    """Uninitialised row_amax [rows] and col_amax [E*K] (fp32)."""
+    return (torch.empty(rows, dtype=torch.float32, device=device),
+            torch.empty(E * K, dtype=torch.float32, device=device))
+
+
+def alloc_outputs(rows: int, K: int, E: int, device="cuda", row: bool = True,
+                  col: bool = True) -> Dict[str, torch.Tensor]:
+    """Uninitialised output buffers of the grouped cast for ``rows`` rows."""
+    out: Dict[str, torch.Tensor] = {}
+    if row:
+        out["row_data"] = torch.empty(rows, K // 2, dtype=torch.uint8, device=device)
+        out["row_scale"] = torch.empty(rows, K // 16, dtype=torch.uint8, device=device)
+        out["row_s2"] = torch.empty(rows, dtype=torch.float32, device=device)
+    if col:
+        out["col_data"] = torch.empty(rows * K // 2, dtype=torch.uint8, device=device)
+        out["col_scale"] = torch.empty(rows * K // 16, dtype=torch.uint8, device=device)
+        out["col_s2"] = torch.empty(E * K, dtype=torch.float32, device=device)
+    return out
+
+
+def routing_tensors(m_splits: Sequence[int], K: int, device="cuda"):
+    """Device first_dims [E] and tensor_offsets [E+1] (element offsets) of a
+    host split list -- the graph-safe routing format."""
+    fd = torch.tensor([int(m) for m in m_splits], dtype=torch.int64)
+    offs = torch.zeros(len(m_splits) + 1, dtype=torch.int64)
+    offs[1:] = torch.cumsum(fd, 0) * K
+    return fd.to(device), offs.to(device)

@@ -1,0 +1,169 @@
+// group_amax.cuh -- grouped amax, both directions from one read of x.
+//
+// TransformerEngine #3649 (grouped row-scaled NVFP4 cast), Description: a
+// single launch over the packed (sum_M, K) bf16 buffer produces the per-row
+// amax [sum_M] and the per-group, per-column amax [E*K]. The per-column amax
+// is what the transposed operand is scaled by (TransformerEngine #3324,
+// summary: columnwise per-column amax).
+//
+// Work split. A 128-row tile always lies inside one group (groups are
+// multiples of 128 rows). The K columns of a tile are split across a
+// thread-block cluster of CN CTAs (CN in {1,2,4,8}, CN divides K/128); each
+// CTA streams its K/CN columns of the tile with 16-byte loads. A CTA's work
+// is cut into units of (128-column chunk, 32-row quarter); warp w takes every
+// unit of quarter w, so the four warps stay balanced for any K.
+//
+// Inside a unit a lane owns 8 columns (one 16-byte chunk) of 16 rows (rows
+// 2i + h of the quarter, h = lane / 16):
+//  - column maxima: packed bf16x2 |.|-max over the lane's 16 rows, merged with
+//    the other half-warp by a shuffle, then into a per-CTA shared array;
+//  - row maxima: the lane's 8-column maximum of each of its 16 rows is
+//    reduced over the 16 lanes sharing those rows with a reduce-scatter
+//    butterfly (8 shuffles), which leaves lane j holding row j's maximum.
+// Row maxima of the CTA's columns meet in shared memory; the cluster's CN
+// partial row maxima are then combined through distributed shared memory by
+// CTA rank 0, which writes row_amax. Column maxima go to col_amax with one
+// unsigned atomic max per column per CTA (non-negative floats order like
+// their bit patterns, and max is order-free, so the result is deterministic).
+// col_amax must be zero before the launch (the host enqueues a memset).
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "codec.cuh"
+#include "routing.cuh"
+
+namespace nvfp4rs {
+
+namespace cg = cooperative_groups;
+
+constexpr int kAmaxThreads = 128;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void red_max_u32(float* addr, uint32_t v) {
+  asm volatile("red.global.max.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+template <class Routing>
+__global__ void __launch_bounds__(kAmaxThreads)
+group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restrict__ x,
+                  int32_t K, int32_t cn, float* __restrict__ row_amax,
+                  float* __restrict__ col_amax) {
+  __shared__ RoutingSmem rs;
+  __shared__ uint32_t rmax[kRows];
+  extern __shared__ uint32_t cmax[];  // [K / cn] column maxima of this CTA (dynamic)
+
+  routing.load(rs);
+
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
+  const int cc = lane & 15, h = lane >> 4;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int tile = blockIdx.x / cn;
+  const int32_t r0 = tile * kRows;
+  const int cols = K / cn;
+  const int c_base = rank * cols;
+  const bool active = rs.ok && r0 < rs.total;
+
+  rmax[t] = 0u;
+  for (int c = t; c < cols; c += kAmaxThreads) cmax[c] = 0u;
+  __syncthreads();
+
+  if (active) {
+    const int nchunks = cols >> 7;
+    const size_t K8 = static_cast<size_t>(K) >> 3;  // row pitch in 16-byte units
+    for (int ch = 0; ch < nchunks; ch++) {
+      // this lane: rows r0 + 32*warp + h + 2i (i < 16), columns c0 .. c0+7
+      const int c_loc = (ch << 7) + (cc << 3);
+      const uint4* p = x + (static_cast<size_t>(r0 + 32 * warp + h) * K8) +
+                       ((c_base + c_loc) >> 3);
+      uint4 v[16];
+#pragma unroll
+      for (int i = 0; i < 16; i++) v[i] = ld_stream(p + 2 * i * K8);
+
+      // column maxima over the lane's 16 rows
+      uint32_t c0 = v[0].x, c1 = v[0].y, c2 = v[0].z, c3 = v[0].w;
+#pragma unroll
+      for (int i = 1; i < 16; i++) {
+        c0 = maxabs2(c0, v[i].x);
+        c1 = maxabs2(c1, v[i].y);
+        c2 = maxabs2(c2, v[i].z);
+        c3 = maxabs2(c3, v[i].w);
+      }
+      // row partial maxima, packed two rows per word: P[k] = (row 2k, row 2k+1)
+      uint32_t P[8];
+#pragma unroll
+      for (int k = 0; k < 8; k++) {
+        const uint32_t a = maxabs2(maxabs2(v[2 * k].x, v[2 * k].y), maxabs2(v[2 * k].z, v[2 * k].w));
+        const uint32_t b = maxabs2(maxabs2(v[2 * k + 1].x, v[2 * k + 1].y),
+                                   maxabs2(v[2 * k + 1].z, v[2 * k + 1].w));
+        // (a.lo, b.lo) vs (a.hi, b.hi)
+        P[k] = maxabs2(prmt(a, b, 0x5410), prmt(a, b, 0x7632)) & 0x7FFF7FFFu;
+      }
+      // reduce-scatter over the 16 lanes of this half-warp: lane cc ends with row cc
+      {
+        const bool b3 = cc & 8, b2 = cc & 4, b1 = cc & 2, b0 = cc & 1;
+        uint32_t Q[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const uint32_t keep = b3 ? P[4 + k] : P[k];
+          const uint32_t send = b3 ? P[k] : P[4 + k];
+          Q[k] = umax2(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 8));
+        }
+        uint32_t R[2];
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+          const uint32_t keep = b2 ? Q[2 + k] : Q[k];
+          const uint32_t send = b2 ? Q[k] : Q[2 + k];
+          R[k] = umax2(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 4));
+        }
+        uint32_t S;
+        {
+          const uint32_t keep = b1 ? R[1] : R[0];
+          const uint32_t send = b1 ? R[0] : R[1];
+          S = umax2(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 2));
+        }
+        const uint32_t keep = b0 ? (S >> 16) : (S & 0xFFFFu);
+        const uint32_t send = b0 ? (S & 0xFFFFu) : (S >> 16);
+        const uint32_t rowm = max(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 1));
+        // lane (cc, h) holds local row 32*warp + h + 2*cc
+        atomicMax(&rmax[32 * warp + h + 2 * cc], rowm << 16);
+      }
+      // merge the two half-warps' column maxima, then into the CTA's array
+      c0 = maxabs2(c0, __shfl_xor_sync(0xFFFFFFFFu, c0, 16)) & 0x7FFF7FFFu;
+      c1 = maxabs2(c1, __shfl_xor_sync(0xFFFFFFFFu, c1, 16)) & 0x7FFF7FFFu;
+      c2 = maxabs2(c2, __shfl_xor_sync(0xFFFFFFFFu, c2, 16)) & 0x7FFF7FFFu;
+      c3 = maxabs2(c3, __shfl_xor_sync(0xFFFFFFFFu, c3, 16)) & 0x7FFF7FFFu;
+      const uint32_t wa = h ? c2 : c0, wb = h ? c3 : c1;  // h=0: cols 0..3, h=1: cols 4..7
+      uint32_t* cm = &cmax[c_loc + 4 * h];
+      atomicMax(cm + 0, wa << 16);
+      atomicMax(cm + 1, wa & 0xFFFF0000u);
+      atomicMax(cm + 2, wb << 16);
+      atomicMax(cm + 3, wb & 0xFFFF0000u);
+    }
+  }
+  __syncthreads();
+  if (active && col_amax != nullptr) {
+    const int g = group_of_row(rs, r0);
+    float* dst = col_amax + static_cast<size_t>(g) * K + c_base;
+    for (int c = t; c < cols; c += kAmaxThreads) red_max_u32(dst + c, cmax[c]);
+  }
+  // every CTA of the cluster reaches both barriers, active or not
+  cluster.sync();
+  if (active && rank == 0 && row_amax != nullptr) {
+    uint32_t m = rmax[t];
+    for (int q = 1; q < cn; q++) m = max(m, *cluster.map_shared_rank(&rmax[t], q));
+    row_amax[r0 + t] = __uint_as_float(m);
+  }
+  cluster.sync();
+}
+
+}  // namespace nvfp4rs

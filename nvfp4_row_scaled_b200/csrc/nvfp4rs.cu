@@ -1,0 +1,269 @@
+// nvfp4rs.cu -- the C ABI of include/nvfp4rs.h: host-side checks, grid
+// shapes and launches of the grouped amax / grouped cast / dequantize kernels.
+//
+// Each public call validates its arguments on the host, then only enqueues
+// memsets and kernels on the caller's stream: no allocation, no
+// synchronisation, no host read of device memory, so every call can be
+// captured in a CUDA graph. The host-split and graph-safe calls instantiate
+// the same kernel templates with a different routing front-end
+// (routing.cuh), which is what makes their outputs byte-identical
+// (TransformerEngine #3649, grouped row-scaled NVFP4 cast, Description).
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "nvfp4rs.h"
+#include "codec.cuh"
+#include "routing.cuh"
+#include "group_amax.cuh"
+#include "group_cast.cuh"
+#include "dequant.cuh"
+
+using namespace nvfp4rs;
+
+namespace {
+
+constexpr int64_t kMaxRows = (int64_t{1} << 31) - kRows;
+constexpr int kMaxAmaxCols = 32768;  // columns per amax CTA (dynamic shared memory)
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+// CTAs per cluster along K for the amax kernel: the largest d <= 8 that
+// divides the number of 128-column chunks.
+int amax_cluster(int64_t K) {
+  const int64_t chunks = K / kCols;
+  for (int d = 8; d > 1; d--)
+    if (chunks % d == 0) return d;
+  return 1;
+}
+
+// Shape checks shared by both steps and both routings.
+nvfp4_status check_shape(const void* x, int64_t rows, int64_t K, int32_t E) {
+  if (rows < 0 || K < 0 || E < 0) return NVFP4_ERR_INVALID_ARG;
+  if (K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows > 0 && K > 0 && x == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (K % kCols != 0 || E > NVFP4_MAX_GROUPS || rows > kMaxRows) return NVFP4_ERR_UNSUPPORTED;
+  if (K / amax_cluster(K) > kMaxAmaxCols) return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned(x, 16)) return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+// Host splits -> HostRouting (row offsets), with the split checks.
+nvfp4_status host_routing(const int64_t* m_splits, int32_t E, int64_t sum_M, HostRouting& r) {
+  if (E > 0 && m_splits == nullptr) return NVFP4_ERR_INVALID_ARG;
+  int64_t total = 0;
+  bool unaligned = false;
+  r.E = E;
+  r.off[0] = 0;
+  for (int32_t g = 0; g < E; g++) {
+    if (m_splits[g] < 0) return NVFP4_ERR_INVALID_ARG;
+    if (m_splits[g] % kRows != 0) unaligned = true;
+    total += m_splits[g];
+    if (total > sum_M) return NVFP4_ERR_INVALID_ARG;
+    r.off[g + 1] = static_cast<int32_t>(total);
+  }
+  if (total != sum_M) return NVFP4_ERR_INVALID_ARG;
+  if (unaligned) return NVFP4_ERR_UNSUPPORTED;
+  r.total = static_cast<int32_t>(total);
+  return NVFP4_OK;
+}
+
+nvfp4_status check_outputs(const nvfp4_outputs* out, bool& do_row, bool& do_col) {
+  if (out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  const int nr = (out->row_data != nullptr) + (out->row_scale != nullptr) + (out->row_s2 != nullptr);
+  const int nc = (out->col_data != nullptr) + (out->col_scale != nullptr) + (out->col_s2 != nullptr);
+  if ((nr != 0 && nr != 3) || (nc != 0 && nc != 3)) return NVFP4_ERR_INVALID_ARG;
+  do_row = nr == 3;
+  do_col = nc == 3;
+  if (!aligned(out->row_data, 16) || !aligned(out->row_scale, 16) || !aligned(out->col_data, 16) ||
+      !aligned(out->col_scale, 16) || !aligned(out->row_s2, 4) || !aligned(out->col_s2, 4))
+    return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+template <class Routing>
+nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t tiles, int64_t K,
+                         float* row_amax, float* col_amax, cudaStream_t stream) {
+  if (tiles == 0 || K == 0) return NVFP4_OK;
+  const int cn = amax_cluster(K);
+  const size_t smem = static_cast<size_t>(K / cn) * sizeof(uint32_t);
+  auto kernel = group_amax_kernel<Routing>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * cn));
+  cfg.blockDim = dim3(kAmaxThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cn);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, static_cast<const uint4*>(x),
+                                        static_cast<int32_t>(K), static_cast<int32_t>(cn),
+                                        row_amax, col_amax));
+}
+
+template <class Routing>
+nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t tiles, int64_t K,
+                         int32_t E, const float* row_amax, const float* col_amax,
+                         const nvfp4_outputs* out, bool do_col, cudaStream_t stream) {
+  const int64_t n_cg = (K / kCols + kColTilesPerCta - 1) / kColTilesPerCta;
+  int64_t n_s2 = 0;
+  if (do_col && E > 0 && K > 0) {
+    n_s2 = (static_cast<int64_t>(E) * K + 4095) / 4096;
+    if (n_s2 > 64) n_s2 = 64;
+  }
+  const int64_t grid = n_s2 + tiles * n_cg;
+  if (grid == 0) return NVFP4_OK;
+  CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kCastThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cuda_status(cudaLaunchKernelEx(&cfg, group_cast_kernel<Routing>, routing,
+                                        static_cast<const uint4*>(x), static_cast<int32_t>(K),
+                                        static_cast<int32_t>(n_cg), static_cast<int32_t>(n_s2),
+                                        row_amax, col_amax, o));
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
+                              const int64_t* m_splits_host, int32_t num_groups, float* row_amax,
+                              float* col_amax, cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  if (sum_M > 0 && row_amax == nullptr && col_amax == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(row_amax, 4) || !aligned(col_amax, 4)) return NVFP4_ERR_UNSUPPORTED;
+  static thread_local HostRouting routing;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  if (s != NVFP4_OK) return s;
+  if (col_amax != nullptr && num_groups > 0 && K > 0) {
+    s = cuda_status(cudaMemsetAsync(col_amax, 0, static_cast<size_t>(num_groups) * K * sizeof(float),
+                                    stream));
+    if (s != NVFP4_OK) return s;
+  }
+  return launch_amax(routing, x_bf16, sum_M / kRows, K, row_amax, col_amax, stream);
+}
+
+nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
+                              const int64_t* m_splits_host, int32_t num_groups,
+                              const float* row_amax, const float* col_amax,
+                              const nvfp4_outputs* out, cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_outputs(out, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  if ((do_row && row_amax == nullptr) || (do_col && col_amax == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  static thread_local HostRouting routing;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  if (s != NVFP4_OK) return s;
+  return launch_cast(routing, x_bf16, sum_M / kRows, K, num_groups, row_amax, col_amax, out,
+                     do_col, stream);
+}
+
+nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                        const int64_t* first_dims_dev,
+                                        const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                        float* row_amax, float* col_amax, int32_t* status_dev,
+                                        cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
+      (num_groups > 0 && first_dims_dev == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (capacity_rows > 0 && row_amax == nullptr && col_amax == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(row_amax, 4) || !aligned(col_amax, 4) || !aligned(status_dev, 4) ||
+      !aligned(first_dims_dev, 8) || !aligned(tensor_offsets_dev, 8))
+    return NVFP4_ERR_UNSUPPORTED;
+  s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
+  if (s != NVFP4_OK) return s;
+  if (col_amax != nullptr && num_groups > 0 && K > 0) {
+    s = cuda_status(cudaMemsetAsync(col_amax, 0, static_cast<size_t>(num_groups) * K * sizeof(float),
+                                    stream));
+    if (s != NVFP4_OK) return s;
+  }
+  if (K == 0) return NVFP4_OK;
+  const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
+                              num_groups};
+  return launch_amax(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, row_amax, col_amax,
+                     stream);
+}
+
+nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                        const int64_t* first_dims_dev,
+                                        const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                        const float* row_amax, const float* col_amax,
+                                        const nvfp4_outputs* out, int32_t* status_dev,
+                                        cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_outputs(out, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  if ((do_row && row_amax == nullptr) || (do_col && col_amax == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
+      (num_groups > 0 && first_dims_dev == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(status_dev, 4) || !aligned(first_dims_dev, 8) || !aligned(tensor_offsets_dev, 8))
+    return NVFP4_ERR_UNSUPPORTED;
+  s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
+  if (s != NVFP4_OK) return s;
+  if (K == 0) return NVFP4_OK;
+  const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
+                              num_groups};
+  return launch_cast(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, num_groups, row_amax,
+                     col_amax, out, do_col, stream);
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
+                              int64_t rows, int64_t cols, float* out_f32, cudaStream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (data == nullptr || scale == nullptr || s2 == nullptr || out_f32 == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(data, 8) || !aligned(out_f32, 16) || !aligned(s2, 4)) return NVFP4_ERR_UNSUPPORTED;
+  const int64_t bpr = cols / 16;
+  const int64_t n = rows * bpr;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t grid = (n + kDequantThreads - 1) / kDequantThreads;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (grid > cap) grid = cap;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kDequantThreads);
+  cfg.stream = stream;
+  return cuda_status(cudaLaunchKernelEx(&cfg, dequant_kernel, reinterpret_cast<const uint2*>(data),
+                                        scale, s2, rows, bpr, reinterpret_cast<float4*>(out_f32)));
+}
+
+const char* nvfp4_status_string(nvfp4_status status) {
+  switch (status) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+    case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    case NVFP4_ERR_ROUTING: return "NVFP4_ERR_ROUTING";
+  }
+  return "NVFP4_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// routing.cuh -- the two routing front-ends of the grouped kernels.
+//
+// TransformerEngine #3649 (grouped row-scaled NVFP4 cast), Description: each
+// of the two steps exists twice, once driven by host split sizes and once by
+// the grouped tensor's device arrays first_dims / tensor_offsets, so that the
+// device-driven pair can be captured in a CUDA graph and replayed after the
+// routing changes; both share one device body, which makes their outputs
+// byte-identical.
+//
+// Here a front-end only fills a RoutingSmem (the first row of every group,
+// the number of groups, the routed row total and a verdict) in shared memory.
+// Everything after that -- which tile belongs to which group, every load,
+// every store -- is the same code for both. The host-split front-end copies
+// the offsets out of the kernel's parameter block; the device front-end loads
+// tensor_offsets / first_dims, checks them, and on a violation records a
+// status code instead of trapping.
+#pragma once
+
+#include <cstdint>
+
+#include "nvfp4rs.h"
+
+namespace nvfp4rs {
+
+constexpr int kRows = 128;  // rows per tile; every group is a multiple of it
+
+struct RoutingSmem {
+  int32_t off[NVFP4_MAX_GROUPS + 1];  // first row of group g; off[E] = routed total
+  int32_t E;
+  int32_t total;
+  int32_t ok;  // 1 when the routing is usable
+};
+
+// Host split sizes turned into row offsets by the host, passed by value.
+struct HostRouting {
+  int32_t E;
+  int32_t total;
+  int32_t off[NVFP4_MAX_GROUPS + 1];
+
+  __device__ __forceinline__ void load(RoutingSmem& s) const {
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) s.off[i] = off[i];
+    if (threadIdx.x == 0) {
+      s.E = E;
+      s.total = total;
+      s.ok = 1;
+    }
+    __syncthreads();
+  }
+};
+
+// Device routing: first_dims [E] rows per group, tensor_offsets [E+1]
+// element offsets (row offset * K). Checked on every load.
+struct DeviceRouting {
+  const int64_t* first_dims;
+  const int64_t* tensor_offsets;
+  int32_t* status;
+  int64_t K;
+  int64_t capacity_rows;
+  int32_t E;
+
+  __device__ __forceinline__ void load(RoutingSmem& s) const {
+    int bad_routing = 0, bad_align = 0;
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+      const int64_t o = tensor_offsets[i];
+      if ((i == 0 && o != 0) || o < 0 || o % K != 0 || o / K > capacity_rows) {
+        bad_routing = 1;
+      } else {
+        s.off[i] = static_cast<int32_t>(o / K);
+      }
+      if (i < E) {
+        const int64_t fd = first_dims[i];
+        const int64_t next = tensor_offsets[i + 1];
+        if (fd < 0 || fd > capacity_rows || next - o != fd * K) bad_routing = 1;
+        if (fd % kRows != 0) bad_align = 1;
+      }
+    }
+    bad_routing = __syncthreads_or(bad_routing);
+    bad_align = __syncthreads_or(bad_align);
+    if (threadIdx.x == 0) {
+      const int code = bad_routing ? NVFP4_ERR_ROUTING : (bad_align ? NVFP4_ERR_UNSUPPORTED : 0);
+      s.E = E;
+      s.ok = code == 0;
+      s.total = code == 0 ? s.off[E] : 0;
+      if (code != 0) *status = code;
+    }
+    __syncthreads();
+  }
+};
+
+// Group holding row r (r < total): the last g with off[g] <= r. Empty groups
+// share their start with the next group and are skipped by taking the last.
+__device__ __forceinline__ int group_of_row(const RoutingSmem& s, int32_t r) {
+  int lo = 0, hi = s.E - 1;  // answer in [lo, hi]
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.off[mid] <= r)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace nvfp4rs

@@ -1,0 +1,126 @@
+"""The C-ABI library, checked without a GPU.
+
+- it builds (nvcc cross-compiles sm_100a here) and loads;
+- it exports every function that include/*.h declares;
+- host-side argument checks return their status before anything is enqueued
+  (none of these calls reaches the CUDA runtime).
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from nvfp4_row_scaled_b200 import abi
+from nvfp4_row_scaled_b200.build import build_library
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_library()
+    return abi.lib()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(nvfp4_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("nvfp4_group_amax", "nvfp4_group_cast", "nvfp4_group_amax_graphsafe",
+                 "nvfp4_group_cast_graphsafe", "nvfp4_dequantize", "nvfp4_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_library_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {abi.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert exported == set(declared_functions()), exported ^ set(declared_functions())
+
+
+def test_status_strings(L):
+    for code, name in [(0, "NVFP4_OK"), (1, "NVFP4_ERR_INVALID_ARG"), (2, "NVFP4_ERR_UNSUPPORTED"),
+                       (3, "NVFP4_ERR_CUDA"), (4, "NVFP4_ERR_ROUTING")]:
+        assert abi.status_name(code) == name
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails its host checks first
+
+
+def amax(L, x, sum_M, K, splits, row=FAKE, col=FAKE):
+    arr = (ctypes.c_int64 * max(len(splits), 1))(*splits) if splits is not None else None
+    return L.nvfp4_group_amax(x, sum_M, K, arr, len(splits or []), row, col, None)
+
+
+@pytest.mark.parametrize("sum_M,K,splits,want", [
+    (256, 24, [256], abi.NVFP4_ERR_INVALID_ARG),       # K % 16
+    (256, 144, [256], abi.NVFP4_ERR_UNSUPPORTED),      # K % 128 (fast path)
+    (256, 128, [128, 64], abi.NVFP4_ERR_INVALID_ARG),  # splits do not add up
+    (256, 128, [384, -128], abi.NVFP4_ERR_INVALID_ARG),  # negative split
+    (192, 128, [64, 128], abi.NVFP4_ERR_UNSUPPORTED),  # group not a multiple of 128
+    (-1, 128, [], abi.NVFP4_ERR_INVALID_ARG),
+])
+def test_amax_host_checks(L, sum_M, K, splits, want):
+    assert amax(L, FAKE, sum_M, K, splits) == want
+
+
+def test_amax_pointer_checks(L):
+    assert amax(L, None, 128, 128, [128]) == abi.NVFP4_ERR_INVALID_ARG
+    assert amax(L, ctypes.c_void_p(0x10008), 128, 128, [128]) == abi.NVFP4_ERR_UNSUPPORTED
+    assert amax(L, FAKE, 128, 128, [128], row=None, col=None) == abi.NVFP4_ERR_INVALID_ARG
+    assert amax(L, FAKE, 128, 128, [128] * (abi.NVFP4_MAX_GROUPS + 1)) == abi.NVFP4_ERR_UNSUPPORTED
+
+
+def test_cast_output_descriptor_checks(L):
+    arr = (ctypes.c_int64 * 1)(128)
+    o = abi.Outputs(row_data=0x10000, row_scale=None, row_s2=0x10000)  # partial direction
+    assert L.nvfp4_group_cast(FAKE, 128, 128, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_INVALID_ARG
+    o = abi.Outputs(row_data=0x10004, row_scale=0x10000, row_s2=0x10000)  # misaligned data
+    assert L.nvfp4_group_cast(FAKE, 128, 128, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_UNSUPPORTED
+    o = abi.Outputs(row_data=0x10000, row_scale=0x10000, row_s2=0x10000)
+    assert L.nvfp4_group_cast(FAKE, 128, 128, arr, 1, None, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_INVALID_ARG  # row direction without row_amax
+    assert L.nvfp4_group_cast(FAKE, 128, 128, arr, 1, FAKE, FAKE, None, None) == \
+        abi.NVFP4_ERR_INVALID_ARG
+
+
+def test_graphsafe_host_checks(L):
+    f = L.nvfp4_group_amax_graphsafe
+    assert f(FAKE, 256, 128, FAKE, FAKE, 2, FAKE, FAKE, None, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 256, 128, FAKE, None, 2, FAKE, FAKE, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 256, 120, FAKE, FAKE, 2, FAKE, FAKE, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 256, 128, ctypes.c_void_p(0x10004), FAKE, 2, FAKE, FAKE, FAKE, None) == \
+        abi.NVFP4_ERR_UNSUPPORTED
+
+
+def test_dequantize_host_checks(L):
+    f = L.nvfp4_dequantize
+    assert f(FAKE, FAKE, FAKE, 4, 24, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, -1, 16, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(None, FAKE, FAKE, 4, 16, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 4, 16, ctypes.c_void_p(0x10008), None) == abi.NVFP4_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 0, 16, FAKE, None) == abi.NVFP4_OK  # empty: nothing to do
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(abi, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(abi, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        abi.lib()
