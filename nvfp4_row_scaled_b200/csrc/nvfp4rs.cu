@@ -71,13 +71,20 @@ nvfp4_status host_routing(const int64_t* m_splits, int32_t E, int64_t sum_M, Hos
   return NVFP4_OK;
 }
 
-nvfp4_status check_outputs(const nvfp4_outputs* out, bool& do_row, bool& do_col) {
+// A direction is requested when any of its three pointers is set; then every
+// one of its buffers that has a nonzero size must be set (a zero-size buffer
+// may be NULL, as allocators hand out for empty tensors).
+nvfp4_status check_outputs(const nvfp4_outputs* out, int64_t rows, int64_t K, int32_t E,
+                           bool& do_row, bool& do_col) {
   if (out == nullptr) return NVFP4_ERR_INVALID_ARG;
-  const int nr = (out->row_data != nullptr) + (out->row_scale != nullptr) + (out->row_s2 != nullptr);
-  const int nc = (out->col_data != nullptr) + (out->col_scale != nullptr) + (out->col_s2 != nullptr);
-  if ((nr != 0 && nr != 3) || (nc != 0 && nc != 3)) return NVFP4_ERR_INVALID_ARG;
-  do_row = nr == 3;
-  do_col = nc == 3;
+  do_row = out->row_data != nullptr || out->row_scale != nullptr || out->row_s2 != nullptr;
+  do_col = out->col_data != nullptr || out->col_scale != nullptr || out->col_s2 != nullptr;
+  const bool has_rows = rows > 0 && K > 0;
+  if (do_row && has_rows && (out->row_data == nullptr || out->row_scale == nullptr || out->row_s2 == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (do_col && ((has_rows && (out->col_data == nullptr || out->col_scale == nullptr)) ||
+                 (E > 0 && K > 0 && out->col_s2 == nullptr)))
+    return NVFP4_ERR_INVALID_ARG;
   if (!aligned(out->row_data, 16) || !aligned(out->row_scale, 16) || !aligned(out->col_data, 16) ||
       !aligned(out->col_scale, 16) || !aligned(out->row_s2, 4) || !aligned(out->col_s2, 4))
     return NVFP4_ERR_UNSUPPORTED;
@@ -168,9 +175,11 @@ nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
   nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
-  s = check_outputs(out, do_row, do_col);
+  s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
   if (s != NVFP4_OK) return s;
-  if ((do_row && row_amax == nullptr) || (do_col && col_amax == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if ((do_row && sum_M > 0 && row_amax == nullptr) ||
+      (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
   static thread_local HostRouting routing;
   s = host_routing(m_splits_host, num_groups, sum_M, routing);
   if (s != NVFP4_OK) return s;
@@ -215,9 +224,11 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
   nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
-  s = check_outputs(out, do_row, do_col);
+  s = check_outputs(out, capacity_rows, K, num_groups, do_row, do_col);
   if (s != NVFP4_OK) return s;
-  if ((do_row && row_amax == nullptr) || (do_col && col_amax == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if ((do_row && capacity_rows > 0 && row_amax == nullptr) ||
+      (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
   if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
       (num_groups > 0 && first_dims_dev == nullptr))
     return NVFP4_ERR_INVALID_ARG;
