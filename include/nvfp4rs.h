@@ -75,7 +75,10 @@ typedef enum {
   NVFP4_ERR_INVALID_ARG = 1, /* null pointer, negative size, splits that do not add up, K % 16 */
   NVFP4_ERR_UNSUPPORTED = 2, /* valid, but outside the fast path (see above) */
   NVFP4_ERR_CUDA = 3,        /* a CUDA call or launch failed */
-  NVFP4_ERR_ROUTING = 4      /* graph-safe only: device routing is inconsistent */
+  NVFP4_ERR_ROUTING = 4,     /* graph-safe only: device routing is inconsistent */
+  NVFP4_ERR_TIMEOUT = 5      /* graph-safe only, device status: a kernel gave up a bounded
+                                wait for its own tile loads (not expected to happen; the
+                                affected outputs are incomplete) */
 } nvfp4_status;
 
 #define NVFP4_MAX_GROUPS 1024

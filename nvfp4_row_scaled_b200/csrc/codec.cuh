@@ -166,3 +166,47 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 }
 
 }  // namespace nvfp4rs
+
+namespace nvfp4rs {
+
+// ------------------------------------------- exact divisions without a divide
+//
+// Markstein's correction (P. Markstein, IBM J. Res. Dev. 34(1), 1990): with
+// y = RN(1/b), q0 = RN(a*y), r = fma(-q0, b, a) (exact), q = fma(r, y, q0)
+// gives q = RN(a/b). The project's tests prove this exhaustively, by exact
+// integer emulation, for every operand pair these two helpers can meet above
+// the 2^-100 cut-off; below it (tiny values, where r could be subnormal) they
+// fall back to the IEEE divide.
+
+// RN(b / 6) for a block maximum b >= 0 (a bf16 value)
+__device__ __forceinline__ float div6(float b) {
+  if (b < 0x1p-100f) return __fdiv_rn(b, 6.0f);
+  const float y = 0x1.555556p-3f;  // RN(1/6)
+  const float q0 = __fmul_rn(b, y);
+  const float r = __fmaf_rn(-q0, 6.0f, b);
+  return __fmaf_rn(r, y, q0);
+}
+
+// Element multiplier min(RN(S / v), FLT_MAX) for S = S_enc and vy = {v,
+// RN(1/v)} of the block's E4M3 scale; vy = {1, 0} for scale code 0 gives 0.
+// An overflowing q0 turns into NaN, which fminf maps to FLT_MAX -- the
+// clamped value of an overflowing quotient.
+__device__ __forceinline__ float elem_scale(float S, float2 vy) {
+  if (S < 0x1p-100f) return vy.y == 0.0f ? 0.0f : fminf(__fdiv_rn(S, vy.x), FLT_MAX);
+  const float q0 = __fmul_rn(S, vy.y);
+  const float r = __fmaf_rn(-q0, vy.x, S);
+  return fminf(__fmaf_rn(r, vy.y, q0), FLT_MAX);
+}
+
+// Table entry for E4M3 code c (0..127): {value, RN(1/value)}; codes 0 and
+// 0x7F (NaN, never produced by the saturating convert) hold {1, 0}.
+__device__ __forceinline__ float2 e4m3_entry(int c) {
+  if (c == 0 || c >= 0x7F) return make_float2(1.0f, 0.0f);
+  const int e = c >> 3, m = c & 7;
+  const float v = e == 0 ? __fmul_rn(static_cast<float>(m), 0x1p-9f)
+                         : __uint_as_float((static_cast<uint32_t>(e + 120) << 23) |
+                                           (static_cast<uint32_t>(m) << 20));
+  return make_float2(v, __frcp_rn(v));
+}
+
+}  // namespace nvfp4rs

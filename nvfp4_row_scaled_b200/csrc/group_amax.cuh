@@ -8,7 +8,7 @@
 //
 // Work split. A 128-row tile always lies inside one group (groups are
 // multiples of 128 rows). The K columns of a tile are split across a
-// thread-block cluster of CN CTAs (CN in {1,2,4,8}, CN divides K/128); each
+// thread-block cluster of CN CTAs (CN <= 8, the largest divisor of K/128); each
 // CTA streams its K/CN columns of the tile with 16-byte loads. A CTA's work
 // is cut into units of (128-column chunk, 32-row quarter); warp w takes every
 // unit of quarter w, so the four warps stay balanced for any K.
@@ -58,9 +58,9 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
                   float* __restrict__ col_amax) {
   __shared__ RoutingSmem rs;
   __shared__ uint32_t rmax[kRows];
-  extern __shared__ uint32_t cmax[];  // [K / cn] column maxima of this CTA (dynamic)
-
-  routing.load(rs);
+  // dynamic: [K / cn] column maxima of this CTA, then the E+1 group offsets
+  extern __shared__ uint32_t cmax[];
+  routing.load(rs, reinterpret_cast<int32_t*>(cmax + K / cn));
 
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;

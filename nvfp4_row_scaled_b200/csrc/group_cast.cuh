@@ -8,23 +8,30 @@
 // scaling; TransformerEngine #3324 (row-scaled backward for GroupedLinear,
 // summary) adds the columnwise (transposed) operand with per-column amax.
 //
-// Work split. A CTA (4 warps) owns one 128-row tile (inside one group) and up
-// to kColTilesPerCta consecutive 128-column tiles of it. For each 128 x 128
-// tile, lane (cc, h) of warp w loads rows 32w + 16h + i (i < 16), columns
-// 8cc .. 8cc+7 with 16-byte loads -- one 16-row x 8-column patch, held in
-// registers. From that patch alone it has:
-//  - 8 complete colwise blocks (16 rows of one column each), and
-//  - 16 half rowwise blocks (8 of 16 columns), completed with lane cc ^ 1.
-// So both directions are encoded from the same registers, with no shared
-// memory transpose of the input. Shared memory only stages the outputs that
-// are not contiguous per lane -- colwise data and scales and rowwise scales
-// -- so that every global store is a full 16- or 8-byte piece of a
-// contiguous run.
-//
-// Extra CTAs at the front of the grid (only when the colwise direction is
-// requested) write col_s2 = S_dec(col_amax) for all E*K entries, empty groups
-// included.
+// Structure (sm_100a):
+//  - Persistent CTAs (two per SM), each walking 128 x 128 tiles of x with a
+//    stride of the grid. A 128-row tile always lies inside one group (groups
+//    are multiples of 128 rows).
+//  - Tiles arrive by TMA: two 2-D tiled loads of 64 columns x 128 rows each
+//    (128-byte rows, 128-byte swizzle, no multicast) into a three-stage
+//    shared-memory ring, completion tracked by one mbarrier per stage. One
+//    thread refills a stage as soon as every thread has read it, so two tiles
+//    are in flight while the third is encoded.
+//  - Lane (cc, h) of warp w reads rows 32w + 16h + i (i < 16), columns
+//    8cc .. 8cc+7 of the tile from shared memory: a 16-row x 8-column patch in
+//    registers that holds 8 complete colwise blocks and 16 half rowwise blocks
+//    (completed with lane cc ^ 1). Both directions are encoded from it.
+//  - Block scales use exact shortcuts instead of IEEE divides: a per-CTA
+//    table of every E4M3 value and its correctly rounded reciprocal, and
+//    Markstein's correction (codec.cuh).
+//  - Outputs that are not contiguous per lane (colwise data and scales,
+//    rowwise scales) are staged in shared memory and stored as full 16- or
+//    8-byte pieces of contiguous runs.
+// Every CTA also writes a slice of col_s2 = S_dec(col_amax) (all E*K
+// entries, empty groups included).
 #pragma once
+
+#include <cuda.h>
 
 #include "codec.cuh"
 #include "routing.cuh"
@@ -32,8 +39,12 @@
 namespace nvfp4rs {
 
 constexpr int kCastThreads = 128;
-constexpr int kColTilesPerCta = 4;
 constexpr int kCols = 128;
+constexpr int kStages = 3;
+constexpr int kBoxCols = 64;                          // TMA box: 64 columns (128 bytes) x 128 rows
+constexpr int kBoxBytes = kBoxCols * kRows * 2;       // 16 KB
+constexpr int kTileBytes = 2 * kBoxBytes;             // 32 KB per 128 x 128 tile
+constexpr uint32_t kSpinLimit = 1u << 22;             // bounded mbarrier waits
 
 struct CastOut {
   uint8_t* row_data;
@@ -44,87 +55,189 @@ struct CastOut {
   float* col_s2;
 };
 
-// Per-tile output staging (one buffer; the kernel double-buffers it).
+// Output staging of one tile.
 struct CastStage {
-  uint8_t col_data[kCols * 64];     // [column][64 B]; 8-byte slot b at (b ^ (column/8 % 8))
-  uint8_t col_scale[8 * kCols];     // [row block][column]
-  uint8_t row_scale[8 * kRows];     // [column block][row]
+  uint8_t col_data[kCols * 64];  // [column][64 B]; 8-byte slot b at (b ^ (column/8 % 8))
+  uint8_t col_scale[8 * kCols];  // [row block][column]
+  uint8_t row_scale[8 * kRows];  // [column block][row]
 };
+
+// Dynamic shared memory of the cast kernel; `off` (E+1 int32) follows it.
+struct CastSmem {
+  uint8_t tile[kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
+  CastStage stage;
+  float2 e4m3[128];                   // {value, RN(1/value)} per E4M3 code
+  float row_senc[kRows];
+  float col_senc[kCols];
+  uint64_t full[kStages];
+};
+
+constexpr size_t cast_smem_bytes(int E) {
+  return ((sizeof(CastSmem) + 15) & ~size_t{15}) + sizeof(int32_t) * (E + 1);
+}
+
+// ------------------------------------------------------------- TMA / mbarrier
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// Wait for the phase with parity `phase` to complete; false after kSpinLimit tries.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
+  const uint32_t a = smem_addr(bar);
+  for (uint32_t i = 0; i < kSpinLimit; i++) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(phase)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Load 128 x 128 tile number `tl` (row tile tl / n_ct, column tile tl % n_ct)
+// into stage s. Both boxes start at a column that is a multiple of 64.
+__device__ __forceinline__ void issue_tile(CastSmem& sm, const CUtensorMap* map, int s, int tl,
+                                           int n_ct) {
+  const int rt = tl / n_ct, ct = tl - rt * n_ct;
+  mbar_expect_tx(&sm.full[s], kTileBytes);
+  tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s]);
+  tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s]);
+}
+
+// ------------------------------------------------------------ block scales
+
+// Block scales of two 16-element blocks (maxima bm0 / bm1, encode scales
+// se0 / se1): the two E4M3 bytes (block 0 in bits 0..7) and the element
+// multipliers S_enc / e4m3(s8) (0 for a zero scale).
+__device__ __forceinline__ uint32_t scales2(float bm0, float se0, float bm1, float se1,
+                                            const float2* tab, float& enc0, float& enc1) {
+  const uint32_t p = e4m3x2(__fmul_rn(div6(bm1), se1), __fmul_rn(div6(bm0), se0));
+  enc0 = elem_scale(se0, tab[p & 0xFFu]);
+  enc1 = elem_scale(se1, tab[p >> 8]);
+  return p;
+}
 
 __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
   *reinterpret_cast<uint32_t*>(p) = v;
 }
 
-template <class Routing>
-__global__ void __launch_bounds__(kCastThreads)
-group_cast_kernel(const __grid_constant__ Routing routing, const uint4* __restrict__ x,
-                  int32_t K, int32_t n_col_groups, int32_t n_s2_ctas,
-                  const float* __restrict__ row_amax, const float* __restrict__ col_amax,
-                  const CastOut out) {
-  __shared__ RoutingSmem rs;
-  __shared__ float row_senc[kRows];
-  __shared__ float col_senc[kColTilesPerCta * kCols];
-  __shared__ __align__(16) CastStage stage[2];
+// ------------------------------------------------------------------ kernel
 
-  routing.load(rs);
+template <class Routing>
+__global__ void __launch_bounds__(kCastThreads, 2)
+group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
+                  int32_t K, const float* __restrict__ row_amax,
+                  const float* __restrict__ col_amax, const CastOut out) {
+  // the 128-byte swizzle wants each stage 1024-byte aligned; the host adds
+  // 1024 bytes of slack for this
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  CastSmem& sm = *reinterpret_cast<CastSmem*>(base);
+  int32_t* off = reinterpret_cast<int32_t*>(base + ((sizeof(CastSmem) + 15) & ~size_t{15}));
+  __shared__ RoutingSmem rs;
+
+  routing.load(rs, off);
   if (!rs.ok) return;
 
   const int t = threadIdx.x;
   const bool do_row = out.row_data != nullptr;
   const bool do_col = out.col_data != nullptr;
 
-  // ---- decode scales of the columns (all groups, empty ones included)
-  if (static_cast<int>(blockIdx.x) < n_s2_ctas) {
+  if (do_col) {  // decode scales of all columns of all groups, spread over the grid
     const int64_t n = static_cast<int64_t>(rs.E) * K;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kCastThreads + t; i < n;
-         i += static_cast<int64_t>(n_s2_ctas) * kCastThreads)
+         i += static_cast<int64_t>(gridDim.x) * kCastThreads)
       out.col_s2[i] = s_dec_of(col_amax[i]);
-    return;
   }
+  sm.e4m3[t] = e4m3_entry(t);
 
-  const int b = blockIdx.x - n_s2_ctas;
-  const int tile = b / n_col_groups;
-  const int cgrp = b % n_col_groups;
-  const int32_t r0 = tile * kRows;
-  if (r0 >= rs.total) return;
-
-  const int g = group_of_row(rs, r0);
-  const int32_t o_g = rs.off[g];
-  const int64_t m_g = rs.off[g + 1] - o_g;
-  const int ct0 = cgrp * kColTilesPerCta;
-  const int nct = min(kColTilesPerCta, (K >> 7) - ct0);
-
-  // ---- second-level scales of this CTA's rows and columns
-  if (do_row) {
-    const float a = row_amax[r0 + t];
-    row_senc[t] = s_enc_of(a);
-    if (cgrp == 0) out.row_s2[r0 + t] = s_dec_of(a);
-  }
-  if (do_col) {
-    const float* ca = col_amax + static_cast<size_t>(g) * K + ct0 * kCols;
-    for (int j = t; j < nct * kCols; j += kCastThreads) col_senc[j] = s_enc_of(ca[j]);
+  const int n_ct = K >> 7;
+  const int n_tiles = (rs.total >> 7) * n_ct;
+  const int G = gridDim.x;
+  if (t == 0) {
+    for (int s = 0; s < kStages; s++) mbar_init(&sm.full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  if (t == 0) {
+    for (int s = 0; s < kStages; s++) {
+      const int tl = blockIdx.x + s * G;
+      if (tl < n_tiles) issue_tile(sm, &tmap, s, tl, n_ct);
+    }
+  }
 
   const int lane = t & 31, warp = t >> 5;
   const int cc = lane & 15, h = lane >> 4;
   const int rb = 2 * warp + h;  // 16-row block of the tile, 0..7
   const int rl = 16 * rb;       // first tile row of this lane
   const bool odd = cc & 1;
-  const size_t K8 = static_cast<size_t>(K) >> 3;
+  CastStage& st = sm.stage;
 
-  for (int j = 0; j < nct; j++) {
-    const int c0 = (ct0 + j) * kCols;
-    CastStage& st = stage[j & 1];
+  int k = 0;
+  bool failed = false;
+  for (int tl = blockIdx.x; tl < n_tiles; tl += G, k++) {
+    const int s = k % kStages;
+    const uint32_t phase = (k / kStages) & 1;
+    const int rt = tl / n_ct, ct = tl - rt * n_ct;
+    const int32_t r0 = rt * kRows;
+    const int c0 = ct * kCols;
+    const int g = group_of_row(rs, r0);
+    const int32_t o_g = rs.off[g];
+    const int64_t m_g = rs.off[g + 1] - o_g;
 
+    // second-level encode scales of this tile's rows and columns
+    if (do_row) {
+      const float a = row_amax[r0 + t];
+      sm.row_senc[t] = s_enc_of(a);
+      if (ct == 0) out.row_s2[r0 + t] = s_dec_of(a);
+    }
+    if (do_col) sm.col_senc[t] = s_enc_of(col_amax[static_cast<size_t>(g) * K + c0 + t]);
+
+    // this lane's 16 x 8 patch from the swizzled stage
+    const bool ok = mbar_wait(&sm.full[s], phase);
     uint4 v[16];
     {
-      const uint4* p = x + static_cast<size_t>(r0 + rl) * K8 + ((c0 >> 3) + cc);
+      const uint8_t* tb = sm.tile[s] + (cc >> 3) * kBoxBytes + rl * 128;
+      const int j = cc & 7;
 #pragma unroll
-      for (int i = 0; i < 16; i++) v[i] = p[i * K8];
+      for (int i = 0; i < 16; i++)
+        v[i] = *reinterpret_cast<const uint4*>(tb + i * 128 + ((j ^ (i & 7)) << 4));
+    }
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    // every thread has read stage s: refill it with this CTA's tile k + kStages
+    if (t == 0 && tl + kStages * G < n_tiles) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue_tile(sm, &tmap, s, tl + kStages * G, n_ct);
     }
 
-    // ---------------------------------------------------- colwise scales
+    // ------------------------------------------------------ colwise scales
     float cenc[8];
     if (do_col) {
       uint32_t m0 = v[0].x, m1 = v[0].y, m2 = v[0].z, m3 = v[0].w;
@@ -137,59 +250,57 @@ group_cast_kernel(const __grid_constant__ Routing routing, const uint4* __restri
       }
       const uint32_t mw[4] = {m0 & 0x7FFF7FFFu, m1 & 0x7FFF7FFFu, m2 & 0x7FFF7FFFu,
                               m3 & 0x7FFF7FFFu};
-      const float* se = &col_senc[j * kCols + 8 * cc];
+      const float* se = &sm.col_senc[8 * cc];
       uint32_t s8w[2] = {0u, 0u};
 #pragma unroll
       for (int q = 0; q < 4; q++) {
-        const uint32_t p2 = block_scales2(bf16lo(mw[q]), se[2 * q], bf16hi(mw[q]), se[2 * q + 1],
-                                          cenc[2 * q], cenc[2 * q + 1]);
+        const uint32_t p2 = scales2(bf16lo(mw[q]), se[2 * q], bf16hi(mw[q]), se[2 * q + 1], sm.e4m3,
+                                    cenc[2 * q], cenc[2 * q + 1]);
         s8w[q >> 1] |= p2 << (16 * (q & 1));
       }
-      // scales of column 8cc+q, row block rb -> col_scale stage [rb][column]
       *reinterpret_cast<uint2*>(&st.col_scale[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
     }
 
-    // ---------------------------------------------------- rowwise scales
+    // ------------------------------------------------------ rowwise scales
     float renc[16];
     if (do_row) {
-      uint32_t P[8];  // (row 2k, row 2k+1) partial maxima over this lane's 8 columns
+      uint32_t P[8];  // (row 2k, row 2k+1) maxima over the whole 16-column block
 #pragma unroll
-      for (int k = 0; k < 8; k++) {
-        const uint32_t a = maxabs2(maxabs2(v[2 * k].x, v[2 * k].y), maxabs2(v[2 * k].z, v[2 * k].w));
-        const uint32_t bb = maxabs2(maxabs2(v[2 * k + 1].x, v[2 * k + 1].y),
-                                    maxabs2(v[2 * k + 1].z, v[2 * k + 1].w));
-        P[k] = maxabs2(prmt(a, bb, 0x5410), prmt(a, bb, 0x7632)) & 0x7FFF7FFFu;
-        P[k] = umax2(P[k], __shfl_xor_sync(0xFFFFFFFFu, P[k], 1));  // whole 16-column block
+      for (int kk = 0; kk < 8; kk++) {
+        const uint32_t a = maxabs2(maxabs2(v[2 * kk].x, v[2 * kk].y), maxabs2(v[2 * kk].z, v[2 * kk].w));
+        const uint32_t b = maxabs2(maxabs2(v[2 * kk + 1].x, v[2 * kk + 1].y),
+                                   maxabs2(v[2 * kk + 1].z, v[2 * kk + 1].w));
+        P[kk] = maxabs2(prmt(a, b, 0x5410), prmt(a, b, 0x7632)) & 0x7FFF7FFFu;
+        P[kk] = umax2(P[kk], __shfl_xor_sync(0xFFFFFFFFu, P[kk], 1));
       }
       // the even lane of a pair scales rows 0..7, the odd lane rows 8..15
       float mine[8];
       uint32_t s8mine[2] = {0u, 0u};
 #pragma unroll
-      for (int k = 0; k < 4; k++) {
-        const uint32_t w = odd ? P[4 + k] : P[k];
-        const int rr = rl + (odd ? 8 : 0) + 2 * k;
-        const uint32_t p2 = block_scales2(bf16lo(w), row_senc[rr], bf16hi(w), row_senc[rr + 1],
-                                          mine[2 * k], mine[2 * k + 1]);
-        s8mine[k >> 1] |= p2 << (16 * (k & 1));
+      for (int kk = 0; kk < 4; kk++) {
+        const uint32_t w = odd ? P[4 + kk] : P[kk];
+        const int rr = rl + (odd ? 8 : 0) + 2 * kk;
+        const uint32_t p2 = scales2(bf16lo(w), sm.row_senc[rr], bf16hi(w), sm.row_senc[rr + 1],
+                                    sm.e4m3, mine[2 * kk], mine[2 * kk + 1]);
+        s8mine[kk >> 1] |= p2 << (16 * (kk & 1));
       }
       float other[8];
 #pragma unroll
-      for (int k = 0; k < 8; k++) other[k] = __shfl_xor_sync(0xFFFFFFFFu, mine[k], 1);
+      for (int kk = 0; kk < 8; kk++) other[kk] = __shfl_xor_sync(0xFFFFFFFFu, mine[kk], 1);
 #pragma unroll
-      for (int k = 0; k < 8; k++) {
-        renc[k] = odd ? other[k] : mine[k];
-        renc[8 + k] = odd ? mine[k] : other[k];
+      for (int kk = 0; kk < 8; kk++) {
+        renc[kk] = odd ? other[kk] : mine[kk];
+        renc[8 + kk] = odd ? mine[kk] : other[kk];
       }
       const uint32_t so0 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[0], 1);
       const uint32_t so1 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[1], 1);
       if (!odd) {
-        // 16 scale bytes of column block cc/2 for rows rl .. rl+15
         *reinterpret_cast<uint4*>(&st.row_scale[(cc >> 1) * kRows + rl]) =
             make_uint4(s8mine[0], s8mine[1], so0, so1);
       }
     }
 
-    // ---------------------------------------------------- codes
+    // -------------------------------------------------------------- codes
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * (K >> 1) + (c0 >> 1) + 4 * cc
                            : nullptr;
     uint32_t cw[2][8];  // colwise words: [rows 0-7 | 8-15][column q]
@@ -200,26 +311,36 @@ group_cast_kernel(const __grid_constant__ Routing routing, const uint4* __restri
       for (int pp = 0; pp < 4; pp++) {
         const int i = 8 * half + 2 * pp;
         const uint4 w0 = v[i], w1 = v[i + 1];
+        const float x0[8] = {bf16lo(w0.x), bf16hi(w0.x), bf16lo(w0.y), bf16hi(w0.y),
+                             bf16lo(w0.z), bf16hi(w0.z), bf16lo(w0.w), bf16hi(w0.w)};
+        const float x1[8] = {bf16lo(w1.x), bf16hi(w1.x), bf16lo(w1.y), bf16hi(w1.y),
+                             bf16lo(w1.z), bf16hi(w1.z), bf16lo(w1.w), bf16hi(w1.w)};
         if (do_row) {
-          st_global_u32(rdst + static_cast<size_t>(i) * (K >> 1), encode_chunk(w0, renc[i]));
-          st_global_u32(rdst + static_cast<size_t>(i + 1) * (K >> 1), encode_chunk(w1, renc[i + 1]));
-        }
-        if (do_col) {
-          const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w};
-          const uint32_t c[4] = {w1.x, w1.y, w1.z, w1.w};
           float y0[8], y1[8];
 #pragma unroll
-          for (int q = 0; q < 4; q++) {
-            mul2(bf16lo(a[q]), bf16hi(a[q]), cenc[2 * q], cenc[2 * q + 1], y0[2 * q], y0[2 * q + 1]);
-            mul2(bf16lo(c[q]), bf16hi(c[q]), cenc[2 * q], cenc[2 * q + 1], y1[2 * q], y1[2 * q + 1]);
+          for (int q = 0; q < 8; q += 2) {
+            mul2(x0[q], x0[q + 1], renc[i], renc[i], y0[q], y0[q + 1]);
+            mul2(x1[q], x1[q + 1], renc[i + 1], renc[i + 1], y1[q], y1[q + 1]);
+          }
+          st_global_u32(rdst + static_cast<size_t>(i) * (K >> 1),
+                        e2m1x8(y0[0], y0[1], y0[2], y0[3], y0[4], y0[5], y0[6], y0[7]));
+          st_global_u32(rdst + static_cast<size_t>(i + 1) * (K >> 1),
+                        e2m1x8(y1[0], y1[1], y1[2], y1[3], y1[4], y1[5], y1[6], y1[7]));
+        }
+        if (do_col) {
+          float y0[8], y1[8];
+#pragma unroll
+          for (int q = 0; q < 8; q += 2) {
+            mul2(x0[q], x0[q + 1], cenc[q], cenc[q + 1], y0[q], y0[q + 1]);
+            mul2(x1[q], x1[q + 1], cenc[q], cenc[q + 1], y1[q], y1[q + 1]);
           }
           // byte q of A = codes of (row i, row i+1) in column q
-          A[pp] = e2m1x2x4(y0[0], y1[0], y0[1], y1[1], y0[2], y1[2], y0[3], y1[3]);
-          B[pp] = e2m1x2x4(y0[4], y1[4], y0[5], y1[5], y0[6], y1[6], y0[7], y1[7]);
+          A[pp] = e2m1x8(y0[0], y1[0], y0[1], y1[1], y0[2], y1[2], y0[3], y1[3]);
+          B[pp] = e2m1x8(y0[4], y1[4], y0[5], y1[5], y0[6], y1[6], y0[7], y1[7]);
         }
       }
       if (do_col) {
-        // 4x4 byte transposes: word for column q = bytes A[0..3][q]
+        // 4x4 byte transposes: the word of column q = bytes A[0..3][q]
         const uint32_t t0 = prmt(A[0], A[1], 0x5140), t1 = prmt(A[0], A[1], 0x7362);
         const uint32_t t2 = prmt(A[2], A[3], 0x5140), t3 = prmt(A[2], A[3], 0x7362);
         cw[half][0] = prmt(t0, t2, 0x5410);
@@ -237,24 +358,23 @@ group_cast_kernel(const __grid_constant__ Routing routing, const uint4* __restri
     if (do_col) {
       const int slot = rb ^ (cc & 7);
 #pragma unroll
-      for (int q = 0; q < 8; q++) {
+      for (int q = 0; q < 8; q++)
         *reinterpret_cast<uint2*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot]) =
             make_uint2(cw[0][q], cw[1][q]);
-      }
     }
     __syncthreads();
 
-    // ---------------------------------------------------- staged stores
+    // ------------------------------------------------------ staged stores
     if (do_col) {
       const size_t half_m = static_cast<size_t>(m_g) >> 1;
       uint8_t* gd = out.col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
 #pragma unroll
-      for (int k = 0; k < 4; k++) {
-        const int u = k * kCastThreads + t;
+      for (int kk = 0; kk < 4; kk++) {
+        const int u = kk * kCastThreads + t;
         const int col = u >> 2, part = u & 3;
-        const int s = (col >> 3) & 7;
-        const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ s)]);
-        const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ s)]);
+        const int sw = (col >> 3) & 7;
+        const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
+        const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
         *reinterpret_cast<uint4*>(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part) =
             make_uint4(lo.x, lo.y, hi.x, hi.y);
       }
@@ -278,6 +398,14 @@ group_cast_kernel(const __grid_constant__ Routing routing, const uint4* __restri
       *reinterpret_cast<uint2*>(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4)) =
           make_uint2(s0, s1);
     }
+  }
+
+  if (failed && t == 0) {
+    // drain the loads this CTA issued and did not consume, then report
+    for (int j = k; j < k + kStages; j++) {
+      if (blockIdx.x + j * G < n_tiles) mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
+    }
+    routing.report(NVFP4_ERR_TIMEOUT);
   }
 }
 

@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cstring>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "nvfp4rs.h"
@@ -47,6 +49,7 @@ nvfp4_status check_shape(const void* x, int64_t rows, int64_t K, int32_t E) {
   if (rows > 0 && K > 0 && x == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (K % kCols != 0 || E > NVFP4_MAX_GROUPS || rows > kMaxRows) return NVFP4_ERR_UNSUPPORTED;
   if (K / amax_cluster(K) > kMaxAmaxCols) return NVFP4_ERR_UNSUPPORTED;
+  if ((rows / kRows) * (K / kCols) > (int64_t{1} << 30)) return NVFP4_ERR_UNSUPPORTED;  // tile ids fit int32
   if (!aligned(x, 16)) return NVFP4_ERR_UNSUPPORTED;
   return NVFP4_OK;
 }
@@ -91,12 +94,41 @@ nvfp4_status check_outputs(const nvfp4_outputs* out, int64_t rows, int64_t K, in
   return NVFP4_OK;
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime (no link to libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// TMA descriptor of x [rows, K] bf16: boxes of 64 columns x 128 rows,
+// 128-byte swizzle (the layout the cast kernel reads back).
+bool x_tensor_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K) {
+  std::memset(map, 0, sizeof(*map));
+  if (rows < kRows || K < kCols) return true;  // no full tile: the map is never used
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBoxCols), static_cast<cuuint32_t>(kRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class Routing>
-nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t tiles, int64_t K,
+nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t tiles, int64_t K, int32_t E,
                          float* row_amax, float* col_amax, cudaStream_t stream) {
   if (tiles == 0 || K == 0) return NVFP4_OK;
   const int cn = amax_cluster(K);
-  const size_t smem = static_cast<size_t>(K / cn) * sizeof(uint32_t);
+  const size_t smem = static_cast<size_t>(K / cn) * sizeof(uint32_t) + sizeof(int32_t) * (E + 1);
   auto kernel = group_amax_kernel<Routing>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -121,29 +153,36 @@ nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t tiles, i
 }
 
 template <class Routing>
-nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t tiles, int64_t K,
-                         int32_t E, const float* row_amax, const float* col_amax,
-                         const nvfp4_outputs* out, bool do_col, cudaStream_t stream) {
-  const int64_t n_cg = (K / kCols + kColTilesPerCta - 1) / kColTilesPerCta;
-  int64_t n_s2 = 0;
-  if (do_col && E > 0 && K > 0) {
-    n_s2 = (static_cast<int64_t>(E) * K + 4095) / 4096;
-    if (n_s2 > 64) n_s2 = 64;
-  }
-  const int64_t grid = n_s2 + tiles * n_cg;
-  if (grid == 0) return NVFP4_OK;
+nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
+                         const float* row_amax, const float* col_amax, const nvfp4_outputs* out,
+                         bool do_col, cudaStream_t stream) {
+  const int64_t tiles = (rows / kRows) * (K / kCols);
+  const bool s2_work = do_col && E > 0 && K > 0;
+  if (tiles == 0 && !s2_work) return NVFP4_OK;
+  CUtensorMap map;
+  if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
+  auto kernel = group_cast_kernel<Routing>;
+  const size_t smem = cast_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCastThreads, smem) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
+  int64_t grid = static_cast<int64_t>(sms) * per_sm;
+  if (tiles > 0 && tiles < grid) grid = tiles;
+  if (grid < 1) grid = 1;
   CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kCastThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
-  return cuda_status(cudaLaunchKernelEx(&cfg, group_cast_kernel<Routing>, routing,
-                                        static_cast<const uint4*>(x), static_cast<int32_t>(K),
-                                        static_cast<int32_t>(n_cg), static_cast<int32_t>(n_s2),
-                                        row_amax, col_amax, o));
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), row_amax,
+                                        col_amax, o));
 }
 
 }  // namespace
@@ -165,7 +204,7 @@ nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
                                     stream));
     if (s != NVFP4_OK) return s;
   }
-  return launch_amax(routing, x_bf16, sum_M / kRows, K, row_amax, col_amax, stream);
+  return launch_amax(routing, x_bf16, sum_M / kRows, K, num_groups, row_amax, col_amax, stream);
 }
 
 nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
@@ -183,8 +222,8 @@ nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
   static thread_local HostRouting routing;
   s = host_routing(m_splits_host, num_groups, sum_M, routing);
   if (s != NVFP4_OK) return s;
-  return launch_cast(routing, x_bf16, sum_M / kRows, K, num_groups, row_amax, col_amax, out,
-                     do_col, stream);
+  return launch_cast(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, out, do_col,
+                     stream);
 }
 
 nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
@@ -211,8 +250,8 @@ nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_row
   if (K == 0) return NVFP4_OK;
   const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
                               num_groups};
-  return launch_amax(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, row_amax, col_amax,
-                     stream);
+  return launch_amax(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, num_groups, row_amax,
+                     col_amax, stream);
 }
 
 nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
@@ -239,8 +278,8 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
   if (K == 0) return NVFP4_OK;
   const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
                               num_groups};
-  return launch_cast(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, num_groups, row_amax,
-                     col_amax, out, do_col, stream);
+  return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
+                     stream);
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
@@ -273,6 +312,7 @@ const char* nvfp4_status_string(nvfp4_status status) {
     case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
     case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
     case NVFP4_ERR_ROUTING: return "NVFP4_ERR_ROUTING";
+    case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
   }
   return "NVFP4_ERR_UNKNOWN";
 }

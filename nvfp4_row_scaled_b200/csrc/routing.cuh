@@ -24,8 +24,10 @@ namespace nvfp4rs {
 
 constexpr int kRows = 128;  // rows per tile; every group is a multiple of it
 
+// Lives in static shared memory; `off` points at E+1 int32 of dynamic shared
+// memory (sized by the host from the number of groups).
 struct RoutingSmem {
-  int32_t off[NVFP4_MAX_GROUPS + 1];  // first row of group g; off[E] = routed total
+  int32_t* off;  // first row of group g; off[E] = routed total
   int32_t E;
   int32_t total;
   int32_t ok;  // 1 when the routing is usable
@@ -37,19 +39,23 @@ struct HostRouting {
   int32_t total;
   int32_t off[NVFP4_MAX_GROUPS + 1];
 
-  __device__ __forceinline__ void load(RoutingSmem& s) const {
-    for (int i = threadIdx.x; i <= E; i += blockDim.x) s.off[i] = off[i];
+  __device__ __forceinline__ void load(RoutingSmem& s, int32_t* off_smem) const {
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off_smem[i] = off[i];
     if (threadIdx.x == 0) {
+      s.off = off_smem;
       s.E = E;
       s.total = total;
       s.ok = 1;
     }
     __syncthreads();
   }
+  // host-split calls have no status word: a give-up is not reported
+  __device__ __forceinline__ void report(int) const {}
 };
 
 // Device routing: first_dims [E] rows per group, tensor_offsets [E+1]
-// element offsets (row offset * K). Checked on every load.
+// element offsets (row offset * K). Checked on every load. `status` is where
+// a violation -- or a kernel's give-up on a bounded wait -- is recorded.
 struct DeviceRouting {
   const int64_t* first_dims;
   const int64_t* tensor_offsets;
@@ -58,14 +64,14 @@ struct DeviceRouting {
   int64_t capacity_rows;
   int32_t E;
 
-  __device__ __forceinline__ void load(RoutingSmem& s) const {
+  __device__ __forceinline__ void load(RoutingSmem& s, int32_t* off_smem) const {
     int bad_routing = 0, bad_align = 0;
     for (int i = threadIdx.x; i <= E; i += blockDim.x) {
       const int64_t o = tensor_offsets[i];
       if ((i == 0 && o != 0) || o < 0 || o % K != 0 || o / K > capacity_rows) {
         bad_routing = 1;
       } else {
-        s.off[i] = static_cast<int32_t>(o / K);
+        off_smem[i] = static_cast<int32_t>(o / K);
       }
       if (i < E) {
         const int64_t fd = first_dims[i];
@@ -78,13 +84,15 @@ struct DeviceRouting {
     bad_align = __syncthreads_or(bad_align);
     if (threadIdx.x == 0) {
       const int code = bad_routing ? NVFP4_ERR_ROUTING : (bad_align ? NVFP4_ERR_UNSUPPORTED : 0);
+      s.off = off_smem;
       s.E = E;
       s.ok = code == 0;
-      s.total = code == 0 ? s.off[E] : 0;
+      s.total = code == 0 ? off_smem[E] : 0;
       if (code != 0) *status = code;
     }
     __syncthreads();
   }
+  __device__ __forceinline__ void report(int code) const { atomicCAS(status, 0, code); }
 };
 
 // Group holding row r (r < total): the last g with off[g] <= r. Empty groups
