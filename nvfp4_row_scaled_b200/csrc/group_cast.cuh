@@ -164,8 +164,10 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   if (!rs.ok) return;
 
   const int t = threadIdx.x;
-  const bool do_row = out.row_data != nullptr;
-  const bool do_col = out.col_data != nullptr;
+  // a requested direction always has its decode-scale buffer (the data and
+  // scale buffers may be NULL only when there are no rows)
+  const bool do_row = out.row_s2 != nullptr;
+  const bool do_col = out.col_s2 != nullptr;
 
   if (do_col) {  // decode scales of all columns of all groups, spread over the grid
     const int64_t n = static_cast<int64_t>(rs.E) * K;
