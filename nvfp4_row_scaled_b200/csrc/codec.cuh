@@ -69,23 +69,6 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float& lo, float& h
       : "=f"(lo), "=f"(hi) : "r"(h2));
 }
 
-// Block scales of two 16-element blocks with maxima bm0 / bm1 and encode
-// scales se0 / se1: returns the two E4M3 bytes (block 0 in bits 0..7) and
-// the element multipliers enc = S_enc / e4m3(s8), 0 when s8 == 0.
-__device__ __forceinline__ uint32_t block_scales2(float bm0, float se0, float bm1, float se1,
-                                                  float& enc0, float& enc1) {
-  const float s0 = __fmul_rn(__fdiv_rn(bm0, 6.0f), se0);
-  const float s1 = __fmul_rn(__fdiv_rn(bm1, 6.0f), se1);
-  const uint32_t p = e4m3x2(s1, s0);
-  float v0, v1;
-  e4m3x2_to_f32(p, v0, v1);
-  const float q0 = fminf(__fdiv_rn(se0, v0), FLT_MAX);
-  const float q1 = fminf(__fdiv_rn(se1, v1), FLT_MAX);
-  enc0 = (p & 0xFFu) ? q0 : 0.0f;
-  enc1 = (p & 0xFF00u) ? q1 : 0.0f;
-  return p;
-}
-
 // ------------------------------------------------------------- E2M1 codes
 
 // d = (a0 * b0, a1 * b1), one IEEE multiply per lane (packed on sm_100a)
@@ -169,35 +152,7 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 
 namespace nvfp4rs {
 
-// ------------------------------------------- exact divisions without a divide
-//
-// Markstein's correction (P. Markstein, IBM J. Res. Dev. 34(1), 1990): with
-// y = RN(1/b), q0 = RN(a*y), r = fma(-q0, b, a) (exact), q = fma(r, y, q0)
-// gives q = RN(a/b). The project's tests prove this exhaustively, by exact
-// integer emulation, for every operand pair these two helpers can meet above
-// the 2^-100 cut-off; below it (tiny values, where r could be subnormal) they
-// fall back to the IEEE divide.
-
-// RN(b / 6) for a block maximum b >= 0 (a bf16 value)
-__device__ __forceinline__ float div6(float b) {
-  if (b < 0x1p-100f) return __fdiv_rn(b, 6.0f);
-  const float y = 0x1.555556p-3f;  // RN(1/6)
-  const float q0 = __fmul_rn(b, y);
-  const float r = __fmaf_rn(-q0, 6.0f, b);
-  return __fmaf_rn(r, y, q0);
-}
-
-// Element multiplier min(RN(S / v), FLT_MAX) for S = S_enc and vy = {v,
-// RN(1/v)} of the block's E4M3 scale; vy = {1, 0} for scale code 0 gives 0.
-// An overflowing q0 turns into NaN, which fminf maps to FLT_MAX -- the
-// clamped value of an overflowing quotient.
-__device__ __forceinline__ float elem_scale(float S, float2 vy) {
-  if (S < 0x1p-100f) return vy.y == 0.0f ? 0.0f : fminf(__fdiv_rn(S, vy.x), FLT_MAX);
-  const float q0 = __fmul_rn(S, vy.y);
-  const float r = __fmaf_rn(-q0, vy.x, S);
-  return fminf(__fmaf_rn(r, vy.y, q0), FLT_MAX);
-}
-
+// E4M3 value table used by the block-scale shortcut below.
 // Table entry for E4M3 code c (0..127): {value, RN(1/value)}; codes 0 and
 // 0x7F (NaN, never produced by the saturating convert) hold {1, 0}.
 __device__ __forceinline__ float2 e4m3_entry(int c) {
@@ -207,6 +162,142 @@ __device__ __forceinline__ float2 e4m3_entry(int c) {
                          : __uint_as_float((static_cast<uint32_t>(e + 120) << 23) |
                                            (static_cast<uint32_t>(m) << 20));
   return make_float2(v, __frcp_rn(v));
+}
+
+}  // namespace nvfp4rs
+
+namespace nvfp4rs {
+
+// --------------------------------------- packed (f32x2) element arithmetic
+//
+// The element path keeps each bf16 pair of a word as one 64-bit register pair
+// (low element in the low half) from the unpack through the multiply to the
+// E2M1 convert, so no moves are needed to form f32x2 operands.
+
+// bf16x2 word -> f32x2 pair (exact)
+__device__ __forceinline__ uint64_t unpack2(uint32_t w) {
+  uint64_t r;
+  asm("{.reg .b32 lo, hi;\n\t"
+      "shl.b32 lo, %1, 16;\n\t"
+      "and.b32 hi, %1, 0xffff0000;\n\t"
+      "mov.b64 %0, {lo, hi};}"
+      : "=l"(r) : "r"(w));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// pairwise IEEE multiply
+__device__ __forceinline__ uint64_t mul2x(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Codes of four pairs, pair i -> byte i with its low element in the low nibble.
+__device__ __forceinline__ uint32_t e2m1_pairs(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
+  uint32_t r;
+  asm("{.reg .b8 b0, b1, b2, b3;\n\t"
+      ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+      "mov.b64 {l0, h0}, %1;\n\t"
+      "mov.b64 {l1, h1}, %2;\n\t"
+      "mov.b64 {l2, h2}, %3;\n\t"
+      "mov.b64 {l3, h3}, %4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, h2, l2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, h3, l3;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};}"
+      : "=r"(r) : "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+  return r;
+}
+
+// Codes across two rows: p (row i) and q (row i+1) hold the same column
+// pair. Byte 0 = (p.lo, q.lo), byte 1 = (p.hi, q.hi), byte 2 = (r.lo, s.lo),
+// byte 3 = (r.hi, s.hi), the row-i value in the low nibble.
+__device__ __forceinline__ uint32_t e2m1_cross(uint64_t p, uint64_t q, uint64_t r, uint64_t s) {
+  uint32_t d;
+  asm("{.reg .b8 b0, b1, b2, b3;\n\t"
+      ".reg .b32 pl, ph, ql, qh, rl, rh, sl, sh;\n\t"
+      "mov.b64 {pl, ph}, %1;\n\t"
+      "mov.b64 {ql, qh}, %2;\n\t"
+      "mov.b64 {rl, rh}, %3;\n\t"
+      "mov.b64 {sl, sh}, %4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, ql, pl;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, qh, ph;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, sl, rl;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, sh, rh;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};}"
+      : "=r"(d) : "l"(p), "l"(q), "l"(r), "l"(s));
+  return d;
+}
+
+// ------------------------------------------------- branch-free block scales
+//
+// Markstein's correction (P. Markstein, IBM J. Res. Dev. 34(1), 1990): with
+// y = RN(1/b), q0 = RN(a*y), r = fma(-q0, b, a) (exact), q = fma(r, y, q0)
+// gives q = RN(a/b). The project's tests prove this exhaustively, by exact
+// integer emulation, for every operand pair used below in its stated range.
+//
+// The common path of a block scale has no branch, so the compiler can
+// interleave the independent blocks of a lane. It is exact whenever the
+// governing (row or column) amax a is 0 or lies in [2^-81, 2^111]:
+//  - then S_enc = 2688 / a >= 2^-100, the range over which the exhaustive
+//    test proves the element-scale shortcut;
+//  - block maxima b >= 2^-100 (or b == 0) are covered by the test of the
+//    divide-by-6 shortcut;
+//  - a block maximum 0 < b < 2^-100 under an amax a >= 2^-81 has
+//    b/6 * 2688/a < 448 * 2^-19 < 2^-10, so its scale is E4M3 zero whether or
+//    not b/6 was rounded exactly, and its multiplier is 0 either way.
+// Tiles holding a row or column outside that range take scales2_exact.
+
+constexpr float kFastAmaxMin = 0x1p-81f;
+constexpr float kFastAmaxMax = 0x1p111f;
+
+__device__ __forceinline__ bool fast_path_amax(float a) {
+  return a == 0.0f || (a >= kFastAmaxMin && a <= kFastAmaxMax);
+}
+
+__device__ __forceinline__ float div6_fast(float b) {
+  const float y = 0x1.555556p-3f;  // RN(1/6)
+  const float q0 = __fmul_rn(b, y);
+  const float r = __fmaf_rn(-q0, 6.0f, b);
+  return __fmaf_rn(r, y, q0);
+}
+
+__device__ __forceinline__ float elem_scale_fast(float S, float2 vy) {
+  const float q0 = __fmul_rn(S, vy.y);
+  const float r = __fmaf_rn(-q0, vy.x, S);
+  return fminf(__fmaf_rn(r, vy.y, q0), FLT_MAX);
+}
+
+__device__ __forceinline__ uint32_t scales2_fast(float bm0, float se0, float bm1, float se1,
+                                                 const float2* tab, float& enc0, float& enc1) {
+  const uint32_t p = e4m3x2(__fmul_rn(div6_fast(bm1), se1), __fmul_rn(div6_fast(bm0), se0));
+  enc0 = elem_scale_fast(se0, tab[p & 0xFFu]);
+  enc1 = elem_scale_fast(se1, tab[p >> 8]);
+  return p;
+}
+
+// The same quantities with IEEE divides (any operand range).
+__device__ __forceinline__ uint32_t scales2_exact(float bm0, float se0, float bm1, float se1,
+                                                  float& enc0, float& enc1) {
+  const uint32_t p = e4m3x2(__fmul_rn(__fdiv_rn(bm1, 6.0f), se1), __fmul_rn(__fdiv_rn(bm0, 6.0f), se0));
+  const float v0 = e4m3_to_f32(p & 0xFFu), v1 = e4m3_to_f32(p >> 8);
+  enc0 = (p & 0xFFu) ? fminf(__fdiv_rn(se0, v0), FLT_MAX) : 0.0f;
+  enc1 = (p & 0xFF00u) ? fminf(__fdiv_rn(se1, v1), FLT_MAX) : 0.0f;
+  return p;
+}
+
+template <bool kExact>
+__device__ __forceinline__ uint32_t scales2_any(float bm0, float se0, float bm1, float se1,
+                                                const float2* tab, float& enc0, float& enc1) {
+  return kExact ? scales2_exact(bm0, se0, bm1, se1, enc0, enc1)
+                : scales2_fast(bm0, se0, bm1, se1, tab, enc0, enc1);
 }
 
 }  // namespace nvfp4rs

@@ -128,21 +128,142 @@ __device__ __forceinline__ void issue_tile(CastSmem& sm, const CUtensorMap* map,
   tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s]);
 }
 
-// ------------------------------------------------------------ block scales
-
-// Block scales of two 16-element blocks (maxima bm0 / bm1, encode scales
-// se0 / se1): the two E4M3 bytes (block 0 in bits 0..7) and the element
-// multipliers S_enc / e4m3(s8) (0 for a zero scale).
-__device__ __forceinline__ uint32_t scales2(float bm0, float se0, float bm1, float se1,
-                                            const float2* tab, float& enc0, float& enc1) {
-  const uint32_t p = e4m3x2(__fmul_rn(div6(bm1), se1), __fmul_rn(div6(bm0), se0));
-  enc0 = elem_scale(se0, tab[p & 0xFFu]);
-  enc1 = elem_scale(se1, tab[p >> 8]);
-  return p;
-}
-
 __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
   *reinterpret_cast<uint32_t*>(p) = v;
+}
+
+// Everything one lane does for one tile after its 16 x 8 patch is in
+// registers: block scales of both directions, all codes, the rowwise data
+// stores and the staging of the other outputs. kExact selects the
+// IEEE-divide block scales (tiles with a row or column amax outside the
+// shortcut's range).
+template <bool kExact>
+__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm, bool do_row,
+                                             bool do_col, int cc, int rb, uint8_t* rdst,
+                                             size_t row_pitch) {
+  const int rl = 16 * rb;
+  const bool odd = cc & 1;
+  CastStage& st = sm.stage;
+
+  // ------------------------------------------------------ colwise scales
+  uint64_t cenc2[4];  // (enc of column 2q, enc of column 2q+1)
+  if (do_col) {
+    uint32_t m0 = v[0].x, m1 = v[0].y, m2 = v[0].z, m3 = v[0].w;
+#pragma unroll
+    for (int i = 1; i < 16; i++) {
+      m0 = maxabs2(m0, v[i].x);
+      m1 = maxabs2(m1, v[i].y);
+      m2 = maxabs2(m2, v[i].z);
+      m3 = maxabs2(m3, v[i].w);
+    }
+    const uint32_t mw[4] = {m0 & 0x7FFF7FFFu, m1 & 0x7FFF7FFFu, m2 & 0x7FFF7FFFu,
+                            m3 & 0x7FFF7FFFu};
+    const float* se = &sm.col_senc[8 * cc];
+    uint32_t s8w[2] = {0u, 0u};
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+      float e0, e1;
+      const uint32_t p2 = scales2_any<kExact>(bf16lo(mw[q]), se[2 * q], bf16hi(mw[q]), se[2 * q + 1],
+                                              sm.e4m3, e0, e1);
+      cenc2[q] = pack2(e0, e1);
+      s8w[q >> 1] |= p2 << (16 * (q & 1));
+    }
+    *reinterpret_cast<uint2*>(&st.col_scale[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
+  }
+
+  // ------------------------------------------------------ rowwise scales
+  uint64_t renc2[16];  // (enc, enc) of row i
+  if (do_row) {
+    uint32_t P[8];  // (row 2k, row 2k+1) maxima over the whole 16-column block
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++) {
+      const uint32_t a = maxabs2(maxabs2(v[2 * kk].x, v[2 * kk].y), maxabs2(v[2 * kk].z, v[2 * kk].w));
+      const uint32_t b = maxabs2(maxabs2(v[2 * kk + 1].x, v[2 * kk + 1].y),
+                                 maxabs2(v[2 * kk + 1].z, v[2 * kk + 1].w));
+      P[kk] = maxabs2(prmt(a, b, 0x5410), prmt(a, b, 0x7632)) & 0x7FFF7FFFu;
+      P[kk] = umax2(P[kk], __shfl_xor_sync(0xFFFFFFFFu, P[kk], 1));
+    }
+    // the even lane of a pair scales rows 0..7, the odd lane rows 8..15
+    float mine[8];
+    uint32_t s8mine[2] = {0u, 0u};
+    const float* rse = &sm.row_senc[rl + (odd ? 8 : 0)];
+#pragma unroll
+    for (int kk = 0; kk < 4; kk++) {
+      const uint32_t w = odd ? P[4 + kk] : P[kk];
+      const uint32_t p2 = scales2_any<kExact>(bf16lo(w), rse[2 * kk], bf16hi(w), rse[2 * kk + 1],
+                                              sm.e4m3, mine[2 * kk], mine[2 * kk + 1]);
+      s8mine[kk >> 1] |= p2 << (16 * (kk & 1));
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++) {
+      const float other = __shfl_xor_sync(0xFFFFFFFFu, mine[kk], 1);
+      const float lo = odd ? other : mine[kk];   // row kk
+      const float hi = odd ? mine[kk] : other;   // row 8 + kk
+      renc2[kk] = pack2(lo, lo);
+      renc2[8 + kk] = pack2(hi, hi);
+    }
+    const uint32_t so0 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[0], 1);
+    const uint32_t so1 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[1], 1);
+    if (!odd) {
+      *reinterpret_cast<uint4*>(&st.row_scale[(cc >> 1) * kRows + rl]) =
+          make_uint4(s8mine[0], s8mine[1], so0, so1);
+    }
+  }
+
+  // -------------------------------------------------------------- codes
+  uint32_t cw[2][8];  // colwise words: [rows 0-7 | 8-15][column q]
+#pragma unroll
+  for (int half = 0; half < 2; half++) {
+    uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
+#pragma unroll
+    for (int pp = 0; pp < 4; pp++) {
+      const int i = 8 * half + 2 * pp;
+      const uint64_t x0[4] = {unpack2(v[i].x), unpack2(v[i].y), unpack2(v[i].z), unpack2(v[i].w)};
+      const uint64_t x1[4] = {unpack2(v[i + 1].x), unpack2(v[i + 1].y), unpack2(v[i + 1].z),
+                              unpack2(v[i + 1].w)};
+      if (do_row) {
+        st_global_u32(rdst + i * row_pitch,
+                      e2m1_pairs(mul2x(x0[0], renc2[i]), mul2x(x0[1], renc2[i]),
+                                 mul2x(x0[2], renc2[i]), mul2x(x0[3], renc2[i])));
+        st_global_u32(rdst + (i + 1) * row_pitch,
+                      e2m1_pairs(mul2x(x1[0], renc2[i + 1]), mul2x(x1[1], renc2[i + 1]),
+                                 mul2x(x1[2], renc2[i + 1]), mul2x(x1[3], renc2[i + 1])));
+      }
+      if (do_col) {
+        uint64_t y0[4], y1[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          y0[q] = mul2x(x0[q], cenc2[q]);
+          y1[q] = mul2x(x1[q], cenc2[q]);
+        }
+        // byte q of A = codes of (row i, row i+1) in column q
+        A[pp] = e2m1_cross(y0[0], y1[0], y0[1], y1[1]);
+        B[pp] = e2m1_cross(y0[2], y1[2], y0[3], y1[3]);
+      }
+    }
+    if (do_col) {
+      // 4x4 byte transposes: the word of column q = bytes A[0..3][q]
+      const uint32_t t0 = prmt(A[0], A[1], 0x5140), t1 = prmt(A[0], A[1], 0x7362);
+      const uint32_t t2 = prmt(A[2], A[3], 0x5140), t3 = prmt(A[2], A[3], 0x7362);
+      cw[half][0] = prmt(t0, t2, 0x5410);
+      cw[half][1] = prmt(t0, t2, 0x7632);
+      cw[half][2] = prmt(t1, t3, 0x5410);
+      cw[half][3] = prmt(t1, t3, 0x7632);
+      const uint32_t u0 = prmt(B[0], B[1], 0x5140), u1 = prmt(B[0], B[1], 0x7362);
+      const uint32_t u2 = prmt(B[2], B[3], 0x5140), u3 = prmt(B[2], B[3], 0x7362);
+      cw[half][4] = prmt(u0, u2, 0x5410);
+      cw[half][5] = prmt(u0, u2, 0x7632);
+      cw[half][6] = prmt(u1, u3, 0x5410);
+      cw[half][7] = prmt(u1, u3, 0x7632);
+    }
+  }
+  if (do_col) {
+    const int slot = rb ^ (cc & 7);
+#pragma unroll
+    for (int q = 0; q < 8; q++)
+      *reinterpret_cast<uint2*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot]) =
+          make_uint2(cw[0][q], cw[1][q]);
+  }
 }
 
 // ------------------------------------------------------------------ kernel
@@ -159,6 +280,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   CastSmem& sm = *reinterpret_cast<CastSmem*>(base);
   int32_t* off = reinterpret_cast<int32_t*>(base + ((sizeof(CastSmem) + 15) & ~size_t{15}));
   __shared__ RoutingSmem rs;
+  __shared__ int slow_tile[2];  // per-tile flag (alternating): some amax outside the shortcut range
 
   routing.load(rs, off);
   if (!rs.ok) return;
@@ -177,47 +299,66 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   }
   sm.e4m3[t] = e4m3_entry(t);
 
+  // this CTA's tiles: a contiguous range of the row-major tile order
   const int n_ct = K >> 7;
   const int n_tiles = (rs.total >> 7) * n_ct;
-  const int G = gridDim.x;
+  const int first = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n_tiles / gridDim.x);
+  const int last = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_tiles / gridDim.x);
   if (t == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&sm.full[s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    slow_tile[0] = 0;
+    slow_tile[1] = 0;
   }
   __syncthreads();
   if (t == 0) {
-    for (int s = 0; s < kStages; s++) {
-      const int tl = blockIdx.x + s * G;
-      if (tl < n_tiles) issue_tile(sm, &tmap, s, tl, n_ct);
-    }
+    for (int s = 0; s < kStages && first + s < last; s++) issue_tile(sm, &tmap, s, first + s, n_ct);
   }
 
   const int lane = t & 31, warp = t >> 5;
   const int cc = lane & 15, h = lane >> 4;
   const int rb = 2 * warp + h;  // 16-row block of the tile, 0..7
   const int rl = 16 * rb;       // first tile row of this lane
-  const bool odd = cc & 1;
+  const size_t row_pitch = static_cast<size_t>(K) >> 1;
   CastStage& st = sm.stage;
 
   int k = 0;
   bool failed = false;
-  for (int tl = blockIdx.x; tl < n_tiles; tl += G, k++) {
+  int cur_rt = -1, rt = 0, ct = 0;
+  bool row_slow = false;
+  int g = 0;
+  int32_t o_g = 0;
+  int64_t m_g = 0;
+  if (first < last) {
+    rt = first / n_ct;
+    ct = first - rt * n_ct;
+  }
+  for (int tl = first; tl < last; tl++, k++) {
     const int s = k % kStages;
     const uint32_t phase = (k / kStages) & 1;
-    const int rt = tl / n_ct, ct = tl - rt * n_ct;
     const int32_t r0 = rt * kRows;
     const int c0 = ct * kCols;
-    const int g = group_of_row(rs, r0);
-    const int32_t o_g = rs.off[g];
-    const int64_t m_g = rs.off[g + 1] - o_g;
-
-    // second-level encode scales of this tile's rows and columns
-    if (do_row) {
-      const float a = row_amax[r0 + t];
-      sm.row_senc[t] = s_enc_of(a);
-      if (ct == 0) out.row_s2[r0 + t] = s_dec_of(a);
+    if (t == 0) slow_tile[(k + 1) & 1] = 0;  // flag of the next tile (last read a tile ago)
+    bool slow = false;
+    if (rt != cur_rt) {  // new row tile: its group and its rows' encode scales
+      cur_rt = rt;
+      g = group_of_row(rs, r0);
+      o_g = rs.off[g];
+      m_g = rs.off[g + 1] - o_g;
+      if (do_row) {
+        const float a = row_amax[r0 + t];
+        sm.row_senc[t] = s_enc_of(a);
+        row_slow = !fast_path_amax(a);
+        if (ct == 0) out.row_s2[r0 + t] = s_dec_of(a);
+      }
     }
-    if (do_col) sm.col_senc[t] = s_enc_of(col_amax[static_cast<size_t>(g) * K + c0 + t]);
+    slow |= row_slow;
+    if (do_col) {
+      const float a = col_amax[static_cast<size_t>(g) * K + c0 + t];
+      sm.col_senc[t] = s_enc_of(a);
+      slow |= !fast_path_amax(a);
+    }
+    if (slow) slow_tile[k & 1] = 1;
 
     // this lane's 16 x 8 patch from the swizzled stage
     const bool ok = mbar_wait(&sm.full[s], phase);
@@ -234,136 +375,17 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
       break;
     }
     // every thread has read stage s: refill it with this CTA's tile k + kStages
-    if (t == 0 && tl + kStages * G < n_tiles) {
+    if (t == 0 && tl + kStages < last) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_tile(sm, &tmap, s, tl + kStages * G, n_ct);
+      issue_tile(sm, &tmap, s, tl + kStages, n_ct);
     }
 
-    // ------------------------------------------------------ colwise scales
-    float cenc[8];
-    if (do_col) {
-      uint32_t m0 = v[0].x, m1 = v[0].y, m2 = v[0].z, m3 = v[0].w;
-#pragma unroll
-      for (int i = 1; i < 16; i++) {
-        m0 = maxabs2(m0, v[i].x);
-        m1 = maxabs2(m1, v[i].y);
-        m2 = maxabs2(m2, v[i].z);
-        m3 = maxabs2(m3, v[i].w);
-      }
-      const uint32_t mw[4] = {m0 & 0x7FFF7FFFu, m1 & 0x7FFF7FFFu, m2 & 0x7FFF7FFFu,
-                              m3 & 0x7FFF7FFFu};
-      const float* se = &sm.col_senc[8 * cc];
-      uint32_t s8w[2] = {0u, 0u};
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const uint32_t p2 = scales2(bf16lo(mw[q]), se[2 * q], bf16hi(mw[q]), se[2 * q + 1], sm.e4m3,
-                                    cenc[2 * q], cenc[2 * q + 1]);
-        s8w[q >> 1] |= p2 << (16 * (q & 1));
-      }
-      *reinterpret_cast<uint2*>(&st.col_scale[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
-    }
-
-    // ------------------------------------------------------ rowwise scales
-    float renc[16];
-    if (do_row) {
-      uint32_t P[8];  // (row 2k, row 2k+1) maxima over the whole 16-column block
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++) {
-        const uint32_t a = maxabs2(maxabs2(v[2 * kk].x, v[2 * kk].y), maxabs2(v[2 * kk].z, v[2 * kk].w));
-        const uint32_t b = maxabs2(maxabs2(v[2 * kk + 1].x, v[2 * kk + 1].y),
-                                   maxabs2(v[2 * kk + 1].z, v[2 * kk + 1].w));
-        P[kk] = maxabs2(prmt(a, b, 0x5410), prmt(a, b, 0x7632)) & 0x7FFF7FFFu;
-        P[kk] = umax2(P[kk], __shfl_xor_sync(0xFFFFFFFFu, P[kk], 1));
-      }
-      // the even lane of a pair scales rows 0..7, the odd lane rows 8..15
-      float mine[8];
-      uint32_t s8mine[2] = {0u, 0u};
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) {
-        const uint32_t w = odd ? P[4 + kk] : P[kk];
-        const int rr = rl + (odd ? 8 : 0) + 2 * kk;
-        const uint32_t p2 = scales2(bf16lo(w), sm.row_senc[rr], bf16hi(w), sm.row_senc[rr + 1],
-                                    sm.e4m3, mine[2 * kk], mine[2 * kk + 1]);
-        s8mine[kk >> 1] |= p2 << (16 * (kk & 1));
-      }
-      float other[8];
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++) other[kk] = __shfl_xor_sync(0xFFFFFFFFu, mine[kk], 1);
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++) {
-        renc[kk] = odd ? other[kk] : mine[kk];
-        renc[8 + kk] = odd ? mine[kk] : other[kk];
-      }
-      const uint32_t so0 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[0], 1);
-      const uint32_t so1 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[1], 1);
-      if (!odd) {
-        *reinterpret_cast<uint4*>(&st.row_scale[(cc >> 1) * kRows + rl]) =
-            make_uint4(s8mine[0], s8mine[1], so0, so1);
-      }
-    }
-
-    // -------------------------------------------------------------- codes
-    uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * (K >> 1) + (c0 >> 1) + 4 * cc
+    uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
                            : nullptr;
-    uint32_t cw[2][8];  // colwise words: [rows 0-7 | 8-15][column q]
-#pragma unroll
-    for (int half = 0; half < 2; half++) {
-      uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
-#pragma unroll
-      for (int pp = 0; pp < 4; pp++) {
-        const int i = 8 * half + 2 * pp;
-        const uint4 w0 = v[i], w1 = v[i + 1];
-        const float x0[8] = {bf16lo(w0.x), bf16hi(w0.x), bf16lo(w0.y), bf16hi(w0.y),
-                             bf16lo(w0.z), bf16hi(w0.z), bf16lo(w0.w), bf16hi(w0.w)};
-        const float x1[8] = {bf16lo(w1.x), bf16hi(w1.x), bf16lo(w1.y), bf16hi(w1.y),
-                             bf16lo(w1.z), bf16hi(w1.z), bf16lo(w1.w), bf16hi(w1.w)};
-        if (do_row) {
-          float y0[8], y1[8];
-#pragma unroll
-          for (int q = 0; q < 8; q += 2) {
-            mul2(x0[q], x0[q + 1], renc[i], renc[i], y0[q], y0[q + 1]);
-            mul2(x1[q], x1[q + 1], renc[i + 1], renc[i + 1], y1[q], y1[q + 1]);
-          }
-          st_global_u32(rdst + static_cast<size_t>(i) * (K >> 1),
-                        e2m1x8(y0[0], y0[1], y0[2], y0[3], y0[4], y0[5], y0[6], y0[7]));
-          st_global_u32(rdst + static_cast<size_t>(i + 1) * (K >> 1),
-                        e2m1x8(y1[0], y1[1], y1[2], y1[3], y1[4], y1[5], y1[6], y1[7]));
-        }
-        if (do_col) {
-          float y0[8], y1[8];
-#pragma unroll
-          for (int q = 0; q < 8; q += 2) {
-            mul2(x0[q], x0[q + 1], cenc[q], cenc[q + 1], y0[q], y0[q + 1]);
-            mul2(x1[q], x1[q + 1], cenc[q], cenc[q + 1], y1[q], y1[q + 1]);
-          }
-          // byte q of A = codes of (row i, row i+1) in column q
-          A[pp] = e2m1x8(y0[0], y1[0], y0[1], y1[1], y0[2], y1[2], y0[3], y1[3]);
-          B[pp] = e2m1x8(y0[4], y1[4], y0[5], y1[5], y0[6], y1[6], y0[7], y1[7]);
-        }
-      }
-      if (do_col) {
-        // 4x4 byte transposes: the word of column q = bytes A[0..3][q]
-        const uint32_t t0 = prmt(A[0], A[1], 0x5140), t1 = prmt(A[0], A[1], 0x7362);
-        const uint32_t t2 = prmt(A[2], A[3], 0x5140), t3 = prmt(A[2], A[3], 0x7362);
-        cw[half][0] = prmt(t0, t2, 0x5410);
-        cw[half][1] = prmt(t0, t2, 0x7632);
-        cw[half][2] = prmt(t1, t3, 0x5410);
-        cw[half][3] = prmt(t1, t3, 0x7632);
-        const uint32_t u0 = prmt(B[0], B[1], 0x5140), u1 = prmt(B[0], B[1], 0x7362);
-        const uint32_t u2 = prmt(B[2], B[3], 0x5140), u3 = prmt(B[2], B[3], 0x7362);
-        cw[half][4] = prmt(u0, u2, 0x5410);
-        cw[half][5] = prmt(u0, u2, 0x7632);
-        cw[half][6] = prmt(u1, u3, 0x5410);
-        cw[half][7] = prmt(u1, u3, 0x7632);
-      }
-    }
-    if (do_col) {
-      const int slot = rb ^ (cc & 7);
-#pragma unroll
-      for (int q = 0; q < 8; q++)
-        *reinterpret_cast<uint2*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot]) =
-            make_uint2(cw[0][q], cw[1][q]);
-    }
+    if (slow_tile[k & 1])
+      encode_patch<true>(v, sm, do_row, do_col, cc, rb, rdst, row_pitch);
+    else
+      encode_patch<false>(v, sm, do_row, do_col, cc, rb, rdst, row_pitch);
     __syncthreads();
 
     // ------------------------------------------------------ staged stores
@@ -400,13 +422,16 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
       *reinterpret_cast<uint2*>(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4)) =
           make_uint2(s0, s1);
     }
+    if (++ct == n_ct) {
+      ct = 0;
+      rt++;
+    }
   }
 
   if (failed && t == 0) {
     // drain the loads this CTA issued and did not consume, then report
-    for (int j = k; j < k + kStages; j++) {
-      if (blockIdx.x + j * G < n_tiles) mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
-    }
+    for (int j = k; j < k + kStages && first + j < last; j++)
+      mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
     routing.report(NVFP4_ERR_TIMEOUT);
   }
 }

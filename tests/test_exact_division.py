@@ -130,3 +130,20 @@ def test_element_scale_over_e4m3():
             assert markstein(am, ae, bm, be, ym, ye) == rn_div(am, ae, bm, be), (s, v)
             n += 1
     assert n > 200000
+
+
+def test_tiny_block_under_fast_range_amax_has_zero_scale():
+    """The kernels use the shortcuts for every block of a tile whose row and
+    column amax values are 0 or in [2^-81, 2^111]. A block maximum below
+    2^-100 is outside the divide-by-6 proof, but under such an amax its
+    block scale is E4M3 zero however b/6 rounds: the largest such scale,
+    from the largest bf16 below 2^-100 under amax 2^-81, is below 2^-10,
+    the smallest value that does not round to E4M3 zero."""
+    b = np.float32(np.uint32(0x0D7F0000).view(np.float32))  # largest bf16 < 2^-100
+    a = np.float32(2.0 ** -81)
+    senc = np.float32(2688.0) / a
+    for t in (np.float32(b / np.float32(6)), np.nextafter(np.float32(b / np.float32(6)), np.float32(1))):
+        s32 = np.float32(t * senc)
+        assert s32 < np.float32(2.0 ** -10) * np.float32(0.9)
+    # and the upper end: S_enc of the largest fast-path amax is still >= 2^-100
+    assert np.float32(2688.0) / np.float32(2.0 ** 111) >= np.float32(2.0 ** -100)
