@@ -9,14 +9,16 @@
 // summary) adds the columnwise (transposed) operand with per-column amax.
 //
 // Structure (sm_100a):
-//  - Persistent CTAs (two per SM), each walking 128 x 128 tiles of x with a
-//    stride of the grid. A 128-row tile always lies inside one group (groups
-//    are multiples of 128 rows).
+//  - Persistent CTAs (three per SM), each taking every gridDim-th 128 x 128
+//    tile of x in row-major tile order, so CTAs running at the same time read
+//    neighbouring tiles of the same rows. A 128-row tile always lies inside
+//    one group (groups are multiples of 128 rows).
 //  - Tiles arrive by TMA: two 2-D tiled loads of 64 columns x 128 rows each
-//    (128-byte rows, 128-byte swizzle, no multicast) into a three-stage
-//    shared-memory ring, completion tracked by one mbarrier per stage. One
-//    thread refills a stage as soon as every thread has read it, so two tiles
-//    are in flight while the third is encoded.
+//    (128-byte rows, 128-byte swizzle, no multicast, L2 evict-first) into a
+//    two-stage shared-memory ring, completion tracked by one mbarrier per
+//    stage. Once every thread holds its patch, the tile's stage is reused to
+//    stage that tile's outputs; it is refilled with the tile after next when
+//    those outputs have been stored.
 //  - Lane (cc, h) of warp w reads rows 32w + 16h + i (i < 16), columns
 //    8cc .. 8cc+7 of the tile from shared memory: a 16-row x 8-column patch in
 //    registers that holds 8 complete colwise blocks and 16 half rowwise blocks
@@ -26,7 +28,9 @@
 //    Markstein's correction (codec.cuh).
 //  - Outputs that are not contiguous per lane (colwise data and scales,
 //    rowwise scales) are staged in shared memory and stored as full 16- or
-//    8-byte pieces of contiguous runs.
+//    8-byte pieces of contiguous runs, with an L2 evict-last hint: a group's
+//    transposed outputs and the 8-byte scale pieces fill their sectors from
+//    several tiles, and should meet in L2 before being written back.
 // Every CTA also writes a slice of col_s2 = S_dec(col_amax) (all E*K
 // entries, empty groups included).
 #pragma once
@@ -40,7 +44,7 @@ namespace nvfp4rs {
 
 constexpr int kCastThreads = 128;
 constexpr int kCols = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kBoxCols = 64;                          // TMA box: 64 columns (128 bytes) x 128 rows
 constexpr int kBoxBytes = kBoxCols * kRows * 2;       // 16 KB
 constexpr int kTileBytes = 2 * kBoxBytes;             // 32 KB per 128 x 128 tile
@@ -65,7 +69,6 @@ struct CastStage {
 // Dynamic shared memory of the cast kernel; `off` (E+1 int32) follows it.
 struct CastSmem {
   uint8_t tile[kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
-  CastStage stage;
   float2 e4m3[128];                   // {value, RN(1/value)} per E4M3 code
   float row_senc[kRows];
   float col_senc[kCols];
@@ -109,12 +112,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
   return false;
 }
 
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void st_global_u2_hint(void* p, uint2 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y),
+               "l"(policy) : "memory");
+}
+__device__ __forceinline__ void st_global_u4_hint(void* p, uint4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy) : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)),
+      "l"(policy_evict_first())
       : "memory");
 }
 
@@ -138,12 +160,11 @@ __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
 // IEEE-divide block scales (tiles with a row or column amax outside the
 // shortcut's range).
 template <bool kExact>
-__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm, bool do_row,
-                                             bool do_col, int cc, int rb, uint8_t* rdst,
-                                             size_t row_pitch) {
+__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm, CastStage& st,
+                                             bool do_row, bool do_col, int cc, int rb,
+                                             uint8_t* rdst, size_t row_pitch) {
   const int rl = 16 * rb;
   const bool odd = cc & 1;
-  CastStage& st = sm.stage;
 
   // ------------------------------------------------------ colwise scales
   uint64_t cenc2[4];  // (enc of column 2q, enc of column 2q+1)
@@ -172,7 +193,7 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
   }
 
   // ------------------------------------------------------ rowwise scales
-  uint64_t renc2[16];  // (enc, enc) of row i
+  float renc[16];  // element multiplier of row i
   if (do_row) {
     uint32_t P[8];  // (row 2k, row 2k+1) maxima over the whole 16-column block
 #pragma unroll
@@ -197,10 +218,8 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
 #pragma unroll
     for (int kk = 0; kk < 8; kk++) {
       const float other = __shfl_xor_sync(0xFFFFFFFFu, mine[kk], 1);
-      const float lo = odd ? other : mine[kk];   // row kk
-      const float hi = odd ? mine[kk] : other;   // row 8 + kk
-      renc2[kk] = pack2(lo, lo);
-      renc2[8 + kk] = pack2(hi, hi);
+      renc[kk] = odd ? other : mine[kk];      // row kk
+      renc[8 + kk] = odd ? mine[kk] : other;  // row 8 + kk
     }
     const uint32_t so0 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[0], 1);
     const uint32_t so1 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[1], 1);
@@ -211,7 +230,7 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
   }
 
   // -------------------------------------------------------------- codes
-  uint32_t cw[2][8];  // colwise words: [rows 0-7 | 8-15][column q]
+  const int slot = rb ^ (cc & 7);
 #pragma unroll
   for (int half = 0; half < 2; half++) {
     uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
@@ -222,12 +241,11 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
       const uint64_t x1[4] = {unpack2(v[i + 1].x), unpack2(v[i + 1].y), unpack2(v[i + 1].z),
                               unpack2(v[i + 1].w)};
       if (do_row) {
-        st_global_u32(rdst + i * row_pitch,
-                      e2m1_pairs(mul2x(x0[0], renc2[i]), mul2x(x0[1], renc2[i]),
-                                 mul2x(x0[2], renc2[i]), mul2x(x0[3], renc2[i])));
-        st_global_u32(rdst + (i + 1) * row_pitch,
-                      e2m1_pairs(mul2x(x1[0], renc2[i + 1]), mul2x(x1[1], renc2[i + 1]),
-                                 mul2x(x1[2], renc2[i + 1]), mul2x(x1[3], renc2[i + 1])));
+        const uint64_t e0 = pack2(renc[i], renc[i]), e1 = pack2(renc[i + 1], renc[i + 1]);
+        st_global_u32(rdst + i * row_pitch, e2m1_pairs(mul2x(x0[0], e0), mul2x(x0[1], e0),
+                                                       mul2x(x0[2], e0), mul2x(x0[3], e0)));
+        st_global_u32(rdst + (i + 1) * row_pitch, e2m1_pairs(mul2x(x1[0], e1), mul2x(x1[1], e1),
+                                                             mul2x(x1[2], e1), mul2x(x1[3], e1)));
       }
       if (do_col) {
         uint64_t y0[4], y1[4];
@@ -242,34 +260,32 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
       }
     }
     if (do_col) {
-      // 4x4 byte transposes: the word of column q = bytes A[0..3][q]
+      // 4x4 byte transposes: the word of column q = bytes A[0..3][q], rows
+      // 8*half .. 8*half+7 of this lane's block, staged right away
+      uint32_t cw[8];
       const uint32_t t0 = prmt(A[0], A[1], 0x5140), t1 = prmt(A[0], A[1], 0x7362);
       const uint32_t t2 = prmt(A[2], A[3], 0x5140), t3 = prmt(A[2], A[3], 0x7362);
-      cw[half][0] = prmt(t0, t2, 0x5410);
-      cw[half][1] = prmt(t0, t2, 0x7632);
-      cw[half][2] = prmt(t1, t3, 0x5410);
-      cw[half][3] = prmt(t1, t3, 0x7632);
+      cw[0] = prmt(t0, t2, 0x5410);
+      cw[1] = prmt(t0, t2, 0x7632);
+      cw[2] = prmt(t1, t3, 0x5410);
+      cw[3] = prmt(t1, t3, 0x7632);
       const uint32_t u0 = prmt(B[0], B[1], 0x5140), u1 = prmt(B[0], B[1], 0x7362);
       const uint32_t u2 = prmt(B[2], B[3], 0x5140), u3 = prmt(B[2], B[3], 0x7362);
-      cw[half][4] = prmt(u0, u2, 0x5410);
-      cw[half][5] = prmt(u0, u2, 0x7632);
-      cw[half][6] = prmt(u1, u3, 0x5410);
-      cw[half][7] = prmt(u1, u3, 0x7632);
-    }
-  }
-  if (do_col) {
-    const int slot = rb ^ (cc & 7);
+      cw[4] = prmt(u0, u2, 0x5410);
+      cw[5] = prmt(u0, u2, 0x7632);
+      cw[6] = prmt(u1, u3, 0x5410);
+      cw[7] = prmt(u1, u3, 0x7632);
 #pragma unroll
-    for (int q = 0; q < 8; q++)
-      *reinterpret_cast<uint2*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot]) =
-          make_uint2(cw[0][q], cw[1][q]);
+      for (int q = 0; q < 8; q++)
+        *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
+    }
   }
 }
 
 // ------------------------------------------------------------------ kernel
 
 template <class Routing>
-__global__ void __launch_bounds__(kCastThreads, 2)
+__global__ void __launch_bounds__(kCastThreads, 3)
 group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
                   int32_t K, const float* __restrict__ row_amax,
                   const float* __restrict__ col_amax, const CastOut out) {
@@ -302,8 +318,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   // this CTA's tiles: a contiguous range of the row-major tile order
   const int n_ct = K >> 7;
   const int n_tiles = (rs.total >> 7) * n_ct;
-  const int first = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n_tiles / gridDim.x);
-  const int last = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_tiles / gridDim.x);
+  const int G = gridDim.x;
   if (t == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&sm.full[s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -312,7 +327,8 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   }
   __syncthreads();
   if (t == 0) {
-    for (int s = 0; s < kStages && first + s < last; s++) issue_tile(sm, &tmap, s, first + s, n_ct);
+    for (int s = 0; s < kStages && blockIdx.x + s * G < n_tiles; s++)
+      issue_tile(sm, &tmap, s, blockIdx.x + s * G, n_ct);
   }
 
   const int lane = t & 31, warp = t >> 5;
@@ -320,22 +336,19 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   const int rb = 2 * warp + h;  // 16-row block of the tile, 0..7
   const int rl = 16 * rb;       // first tile row of this lane
   const size_t row_pitch = static_cast<size_t>(K) >> 1;
-  CastStage& st = sm.stage;
 
   int k = 0;
   bool failed = false;
-  int cur_rt = -1, rt = 0, ct = 0;
+  int cur_rt = -1;
   bool row_slow = false;
   int g = 0;
   int32_t o_g = 0;
   int64_t m_g = 0;
-  if (first < last) {
-    rt = first / n_ct;
-    ct = first - rt * n_ct;
-  }
-  for (int tl = first; tl < last; tl++, k++) {
+  const uint64_t keep = policy_evict_last();
+  for (int tl = blockIdx.x; tl < n_tiles; tl += G, k++) {
     const int s = k % kStages;
     const uint32_t phase = (k / kStages) & 1;
+    const int rt = tl / n_ct, ct = tl - rt * n_ct;
     const int32_t r0 = rt * kRows;
     const int c0 = ct * kCols;
     if (t == 0) slow_tile[(k + 1) & 1] = 0;  // flag of the next tile (last read a tile ago)
@@ -374,18 +387,21 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
       failed = true;
       break;
     }
-    // every thread has read stage s: refill it with this CTA's tile k + kStages
-    if (t == 0 && tl + kStages < last) {
+    // The other stage held tile k-1, whose staged outputs were stored before
+    // this barrier: refill it with tile k+1 (tiles 0 and 1 came in the prologue).
+    if (t == 0 && k >= 1 && tl + G < n_tiles) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_tile(sm, &tmap, s, tl + kStages, n_ct);
+      issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
     }
+    // stage s is free once every thread holds its patch: it stages the outputs
+    CastStage& st = *reinterpret_cast<CastStage*>(sm.tile[s]);
 
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
                            : nullptr;
     if (slow_tile[k & 1])
-      encode_patch<true>(v, sm, do_row, do_col, cc, rb, rdst, row_pitch);
+      encode_patch<true>(v, sm, st, do_row, do_col, cc, rb, rdst, row_pitch);
     else
-      encode_patch<false>(v, sm, do_row, do_col, cc, rb, rdst, row_pitch);
+      encode_patch<false>(v, sm, st, do_row, do_col, cc, rb, rdst, row_pitch);
     __syncthreads();
 
     // ------------------------------------------------------ staged stores
@@ -399,8 +415,8 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
         const int sw = (col >> 3) & 7;
         const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
         const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
-        *reinterpret_cast<uint4*>(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part) =
-            make_uint4(lo.x, lo.y, hi.x, hi.y);
+        st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part,
+                          make_uint4(lo.x, lo.y, hi.x, hi.y), keep);
       }
       const size_t m16 = static_cast<size_t>(m_g) >> 4;
       uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
@@ -410,7 +426,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
         s0 |= static_cast<uint32_t>(st.col_scale[r * kCols + t]) << (8 * r);
         s1 |= static_cast<uint32_t>(st.col_scale[(r + 4) * kCols + t]) << (8 * r);
       }
-      *reinterpret_cast<uint2*>(gs + static_cast<size_t>(c0 + t) * m16) = make_uint2(s0, s1);
+      st_global_u2_hint(gs + static_cast<size_t>(c0 + t) * m16, make_uint2(s0, s1), keep);
     }
     if (do_row) {
       uint32_t s0 = 0u, s1 = 0u;
@@ -419,18 +435,15 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
         s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
         s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
       }
-      *reinterpret_cast<uint2*>(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4)) =
-          make_uint2(s0, s1);
-    }
-    if (++ct == n_ct) {
-      ct = 0;
-      rt++;
+      st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
+                        make_uint2(s0, s1), keep);
     }
   }
 
   if (failed && t == 0) {
-    // drain the loads this CTA issued and did not consume, then report
-    for (int j = k; j < k + kStages && first + j < last; j++)
+    // drain the loads this CTA issued and did not consume (tile k, and tile 1
+    // when the prologue's second load is still outstanding), then report
+    for (int j = k; j <= (k == 0 ? 1 : k) && blockIdx.x + j * G < n_tiles; j++)
       mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
     routing.report(NVFP4_ERR_TIMEOUT);
   }
