@@ -89,6 +89,24 @@ def traffic_record(kernel: str, workload: str):
     return r.get("bytes_per_launch")
 
 
+# ----------------------------------------------------------- multi-rank
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The job's time is the slowest rank's: all-reduce(MAX) when world > 1."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(elements_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job Gelem/s: every rank casts its own batch (weak scaling)."""
+    return world * elements_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -270,10 +288,7 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_end)
     amax_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     cast_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     # ---- end to end through the C ABI with host buffers (pinned)
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
@@ -292,10 +307,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
 
     if world > 1:
         dist.destroy_process_group()
@@ -303,7 +315,7 @@ def main():
         return
 
     ms_per_step = elapsed_ms / args.steps
-    value = world * N / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(N, world, ms_per_step)
     b = algorithmic_bytes(M, K, E)
     peak, peak_kind = hbm_peak()
     dominant = "cast" if cast_ms >= amax_ms else "amax"
@@ -354,7 +366,7 @@ def main():
         },
         "cpu_baseline": cpu,
         "e2e": {
-            "value": round(world * N / (e2e_ms * 1e-3) / 1e9, 3),
+            "value": round(job_throughput(N, world, e2e_ms), 3),
             "unit": "Gelem/s",
             "h2d_bytes_per_step": 2 * N,
             "d2h_bytes_per_step": output_bytes(M, K, E),
