@@ -7,11 +7,13 @@
 // summary: columnwise per-column amax).
 //
 // Work split. A 128-row tile always lies inside one group (groups are
-// multiples of 128 rows). The K columns of a tile are split across a
-// thread-block cluster of CN CTAs (CN <= 8, the largest divisor of K/128); each
-// CTA streams its K/CN columns of the tile with 16-byte loads. A CTA's work
-// is cut into units of (128-column chunk, 32-row quarter); warp w takes every
-// unit of quarter w, so the four warps stay balanced for any K.
+// multiples of 128 rows). The K/128 column chunks of a tile are dealt round
+// robin to a thread-block cluster of CN CTAs (CN <= 8, the largest divisor of
+// K/128): CTA q takes chunks q, q + CN, q + 2CN, ..., so the cluster reads each
+// row left to right in CN * 256-byte runs (much kinder to DRAM than one slab
+// per CTA). A CTA's work is cut into units of (128-column chunk, 32-row
+// quarter); warp w takes every unit of quarter w, so the four warps stay
+// balanced for any K.
 //
 // Inside a unit a lane owns 8 columns (one 16-byte chunk) of 16 rows (rows
 // 2i + h of the quarter, h = lane / 16):
@@ -70,7 +72,6 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   const int tile = blockIdx.x / cn;
   const int32_t r0 = tile * kRows;
   const int cols = K / cn;
-  const int c_base = rank * cols;
   const bool active = rs.ok && r0 < rs.total;
 
   rmax[t] = 0u;
@@ -82,9 +83,9 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
     const size_t K8 = static_cast<size_t>(K) >> 3;  // row pitch in 16-byte units
     for (int ch = 0; ch < nchunks; ch++) {
       // this lane: rows r0 + 32*warp + h + 2i (i < 16), columns c0 .. c0+7
-      const int c_loc = (ch << 7) + (cc << 3);
-      const uint4* p = x + (static_cast<size_t>(r0 + 32 * warp + h) * K8) +
-                       ((c_base + c_loc) >> 3);
+      const int c_loc = (ch << 7) + (cc << 3);                // index into this CTA's cmax
+      const int c_glb = ((ch * cn + rank) << 7) + (cc << 3);  // chunk ch of the CTA: rank + ch*cn
+      const uint4* p = x + (static_cast<size_t>(r0 + 32 * warp + h) * K8) + (c_glb >> 3);
       uint4 v[16];
 #pragma unroll
       for (int i = 0; i < 16; i++) v[i] = ld_stream(p + 2 * i * K8);
@@ -153,8 +154,9 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   __syncthreads();
   if (active && col_amax != nullptr) {
     const int g = group_of_row(rs, r0);
-    float* dst = col_amax + static_cast<size_t>(g) * K + c_base;
-    for (int c = t; c < cols; c += kAmaxThreads) red_max_u32(dst + c, cmax[c]);
+    float* dst = col_amax + static_cast<size_t>(g) * K;
+    for (int c = t; c < cols; c += kAmaxThreads)
+      red_max_u32(dst + ((((c >> 7) * cn + rank) << 7) | (c & 127)), cmax[c]);
   }
   // every CTA of the cluster reaches both barriers, active or not
   cluster.sync();
