@@ -290,6 +290,23 @@ def main():
     cast_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
+    # ---- the one-launch path (amax + cast in one persistent kernel), same
+    # workload and outputs, timed the same way (reported beside the headline)
+    ws = abi.alloc_workspace(0, E, dev)
+    for _ in range(args.warmup):
+        abi.nvfp4_group_quantize(x, splits, ra, ca, out, ws)
+    torch.cuda.synchronize(dev)
+    barrier()
+    q0 = torch.cuda.Event(enable_timing=True)
+    q1 = torch.cuda.Event(enable_timing=True)
+    q0.record(stream)
+    for _ in range(args.steps):
+        abi.nvfp4_group_quantize(x, splits, ra, ca, out, ws)
+    q1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    one_ms = max_over_ranks(q0.elapsed_time(q1) / args.steps, world, dev)
+
     # ---- end to end through the C ABI with host buffers (pinned)
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
     e2e_steps = max(3, min(args.steps, 5))
@@ -370,6 +387,15 @@ def main():
             "unit": "Gelem/s",
             "h2d_bytes_per_step": 2 * N,
             "d2h_bytes_per_step": output_bytes(M, K, E),
+        },
+        "one_launch": {
+            "path": "nvfp4_group_quantize (grouped amax + cast in one persistent kernel)",
+            "value": round(job_throughput(N, world, one_ms), 3),
+            "unit": "Gelem/s",
+            "ms_per_step": round(one_ms, 4),
+            "hbm_gbs": round(b["cast"] / (one_ms * 1e-3) / 1e9, 1),
+            "hbm_frac_of_peak": round(b["cast"] / (one_ms * 1e-3) / 1e9 / peak, 4),
+            "algorithmic_bytes_per_launch": b["cast"],
         },
         "gpu_launches": 2 * args.steps,
         "clocks": clk,

@@ -62,6 +62,7 @@
 #ifndef NVFP4RS_H
 #define NVFP4RS_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #include <cuda_runtime_api.h> /* cudaStream_t */
@@ -77,7 +78,8 @@ typedef enum {
   NVFP4_ERR_CUDA = 3,        /* a CUDA call or launch failed */
   NVFP4_ERR_ROUTING = 4,     /* graph-safe only: device routing is inconsistent */
   NVFP4_ERR_TIMEOUT = 5      /* graph-safe only, device status: a kernel gave up a bounded
-                                wait for its own tile loads (not expected to happen; the
+                                wait for its own tile loads or, in the one-launch call, for
+                                another CTA's amax work (not expected to happen; the
                                 affected outputs are incomplete) */
 } nvfp4_status;
 
@@ -177,6 +179,63 @@ NVFP4RS_API nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t 
                                         const float* row_amax, const float* col_amax,
                                         const nvfp4_outputs* out, int32_t* status_dev,
                                         cudaStream_t stream);
+
+/*
+ * Bytes of workspace the one-launch calls below need. The graph-safe call
+ * needs nvfp4_group_quantize_workspace_bytes(capacity_rows, num_groups); the
+ * host-split call needs only nvfp4_group_quantize_workspace_bytes(0,
+ * num_groups) (at most 4352 bytes). Returns 0 for a negative size or
+ * num_groups > NVFP4_MAX_GROUPS.
+ */
+NVFP4RS_API size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, int32_t num_groups);
+
+/*
+ * Grouped amax AND grouped cast in ONE launch, host-split routing. Computes
+ * exactly what nvfp4_group_amax followed by nvfp4_group_cast computes
+ * (TransformerEngine #3649, Description: the amax step's row and column amax
+ * vectors are the cast step's scale sources) -- row_amax, col_amax and every
+ * output of `out` byte-identical to that pair -- but reads each tile of x
+ * from DRAM once: a persistent kernel runs the amax of a tile, and the cast
+ * of the same tile a little later while it is still in L2, once all amax
+ * work of its group has finished.
+ *   x_bf16, sum_M, K, m_splits_host, num_groups, out
+ *                   as for nvfp4_group_cast
+ *   row_amax        device fp32 [sum_M], written (needed when the row
+ *                   direction is requested, else may be NULL)
+ *   col_amax        device fp32 [num_groups*K], written (needed when the
+ *                   column direction is requested, else may be NULL)
+ *   workspace       device, >= nvfp4_group_quantize_workspace_bytes(0,
+ *                   num_groups) bytes, 16-byte aligned, owned by the caller;
+ *                   zeroed by this call on `stream`, so calls that share a
+ *                   workspace must be ordered on one stream. After the call
+ *                   word 1 is nonzero only if a bounded wait inside the kernel
+ *                   gave up (not expected; the outputs are then incomplete).
+ * With no direction requested nothing is enqueued. Memsets of the workspace
+ * header, row_amax and col_amax, then one launch.
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
+                                  const int64_t* m_splits_host, int32_t num_groups,
+                                  float* row_amax, float* col_amax, const nvfp4_outputs* out,
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * nvfp4_group_quantize with the graph-safe routing of
+ * nvfp4_group_amax_graphsafe (same routing arguments and status rules, plus
+ * NVFP4_ERR_TIMEOUT if a bounded wait gave up). Byte-identical to the
+ * host-split call for equal routing, and to the graph-safe two-launch pair.
+ * Rows at or beyond the routed total are neither read nor written; their row
+ * amax accumulates in the workspace, which must hold
+ * nvfp4_group_quantize_workspace_bytes(capacity_rows, num_groups) bytes.
+ * Memsets of status, the workspace and col_amax, then one launch; capturable
+ * in a CUDA graph.
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                            const int64_t* first_dims_dev,
+                                            const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                            float* row_amax, float* col_amax,
+                                            const nvfp4_outputs* out, void* workspace,
+                                            size_t workspace_bytes, int32_t* status_dev,
+                                            cudaStream_t stream);
 
 /*
  * Dequantize one quantized matrix [rows, cols] to FP32 with one decode scale

@@ -30,6 +30,7 @@ NVFP4_ERR_INVALID_ARG = 1
 NVFP4_ERR_UNSUPPORTED = 2
 NVFP4_ERR_CUDA = 3
 NVFP4_ERR_ROUTING = 4
+NVFP4_ERR_TIMEOUT = 5
 NVFP4_MAX_GROUPS = 1024
 
 _lib = None
@@ -63,8 +64,16 @@ def lib():
         L.nvfp4_group_cast_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp,
                                                  ctypes.POINTER(Outputs), vp, vp]
         L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, vp]
+        sz = ctypes.c_size_t
+        L.nvfp4_group_quantize_workspace_bytes.argtypes = [i64, i32]
+        L.nvfp4_group_quantize_workspace_bytes.restype = sz
+        L.nvfp4_group_quantize.argtypes = [vp, i64, i64, vp, i32, vp, vp, ctypes.POINTER(Outputs),
+                                           vp, sz, vp]
+        L.nvfp4_group_quantize_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp,
+                                                     ctypes.POINTER(Outputs), vp, sz, vp, vp]
         for f in ("nvfp4_group_amax", "nvfp4_group_cast", "nvfp4_group_amax_graphsafe",
-                  "nvfp4_group_cast_graphsafe", "nvfp4_dequantize"):
+                  "nvfp4_group_cast_graphsafe", "nvfp4_dequantize", "nvfp4_group_quantize",
+                  "nvfp4_group_quantize_graphsafe"):
             getattr(L, f).restype = ctypes.c_int
         L.nvfp4_status_string.argtypes = [ctypes.c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
@@ -164,6 +173,45 @@ def nvfp4_group_cast_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
     _check(rc, "nvfp4_group_cast_graphsafe")
 
 
+def nvfp4_group_quantize_workspace_bytes(capacity_rows: int, num_groups: int) -> int:
+    return int(lib().nvfp4_group_quantize_workspace_bytes(int(capacity_rows), int(num_groups)))
+
+
+def _workspace(ws: torch.Tensor):
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+
+def nvfp4_group_quantize(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optional[torch.Tensor],
+                         col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
+                         workspace: torch.Tensor, stream=None) -> None:
+    arr, E = _splits(m_splits)
+    o = _outputs(out)
+    wp, wb = _workspace(workspace)
+    rc = lib().nvfp4_group_quantize(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
+                                    _dev(row_amax, torch.float32, "row_amax"),
+                                    _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
+                                    wp, wb, _stream(stream))
+    _check(rc, "nvfp4_group_quantize")
+
+
+def nvfp4_group_quantize_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
+                                   tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
+                                   col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
+                                   workspace: torch.Tensor, status: torch.Tensor,
+                                   stream=None) -> None:
+    o = _outputs(out)
+    wp, wb = _workspace(workspace)
+    rc = lib().nvfp4_group_quantize_graphsafe(
+        _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
+        _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
+        first_dims.numel(), _dev(row_amax, torch.float32, "row_amax"),
+        _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o), wp, wb,
+        _dev(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "nvfp4_group_quantize_graphsafe")
+
+
 def nvfp4_dequantize(data: torch.Tensor, scale: torch.Tensor, s2: torch.Tensor, rows: int, cols: int,
                      out: torch.Tensor, stream=None) -> None:
     rc = lib().nvfp4_dequantize(_dev(data, torch.uint8, "data"), _dev(scale, torch.uint8, "scale"),
@@ -193,6 +241,13 @@ def alloc_outputs(rows: int, K: int, E: int, device="cuda", row: bool = True,
         out["col_scale"] = torch.empty(rows * K // 16, dtype=torch.uint8, device=device)
         out["col_s2"] = torch.empty(E * K, dtype=torch.float32, device=device)
     return out
+
+
+def alloc_workspace(capacity_rows: int, num_groups: int, device="cuda") -> torch.Tensor:
+    """Workspace of the one-launch calls (uint8; its contents need no
+    initialisation, the calls zero what they use)."""
+    return torch.empty(nvfp4_group_quantize_workspace_bytes(capacity_rows, num_groups),
+                       dtype=torch.uint8, device=device)
 
 
 def routing_tensors(m_splits: Sequence[int], K: int, device="cuda"):

@@ -95,10 +95,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
-// Wait for the phase with parity `phase` to complete; false after kSpinLimit tries.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
+// Wait for the phase with parity `phase` to complete; false after `tries` tries.
+__device__ __forceinline__ bool mbar_wait_some(uint64_t* bar, uint32_t phase, uint32_t tries) {
   const uint32_t a = smem_addr(bar);
-  for (uint32_t i = 0; i < kSpinLimit; i++) {
+  for (uint32_t i = 0; i < tries; i++) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -110,6 +110,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
     if (done) return true;
   }
   return false;
+}
+
+// Wait for the phase with parity `phase` to complete; false after kSpinLimit tries.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
+  return mbar_wait_some(bar, phase, kSpinLimit);
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -130,24 +135,45 @@ __device__ __forceinline__ void st_global_u4_hint(void* p, uint4 v, uint64_t pol
   asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy) : "memory");
 }
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
+                                            uint64_t* bar, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)),
-      "l"(policy_evict_first())
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
 
-// Load 128 x 128 tile number `tl` (row tile tl / n_ct, column tile tl % n_ct)
-// into stage s. Both boxes start at a column that is a multiple of 64.
+// Load the 128 x 128 tile (row tile rt, column tile ct) into stage s. Both
+// boxes start at a column that is a multiple of 64 (128 bytes).
+__device__ __forceinline__ void issue_tile_at(CastSmem& sm, const CUtensorMap* map, int s, int rt,
+                                              int ct, uint64_t policy) {
+  mbar_expect_tx(&sm.full[s], kTileBytes);
+  tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s], policy);
+  tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s], policy);
+}
+
+// Tile number `tl` of the row-major tile order (read once: evict first).
 __device__ __forceinline__ void issue_tile(CastSmem& sm, const CUtensorMap* map, int s, int tl,
                                            int n_ct) {
-  const int rt = tl / n_ct, ct = tl - rt * n_ct;
-  mbar_expect_tx(&sm.full[s], kTileBytes);
-  tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s]);
-  tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s]);
+  const int rt = tl / n_ct;
+  issue_tile_at(sm, map, s, rt, tl - rt * n_ct, policy_evict_first());
+}
+
+// Lane (cc, h) of warp w: rows rl .. rl+15 (rl = 16 * (2w + h)), columns
+// 8cc .. 8cc+7 of the swizzled 128 x 128 tile at `tile` (two 64-column boxes).
+__device__ __forceinline__ void load_patch(const uint8_t* tile, int cc, int rl, uint4 (&v)[16]) {
+  const uint8_t* tb = tile + (cc >> 3) * kBoxBytes + rl * 128;
+  const int j = cc & 7;
+#pragma unroll
+  for (int i = 0; i < 16; i++)
+    v[i] = *reinterpret_cast<const uint4*>(tb + i * 128 + ((j ^ (i & 7)) << 4));
 }
 
 __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
@@ -159,8 +185,16 @@ __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
 // stores and the staging of the other outputs. kExact selects the
 // IEEE-divide block scales (tiles with a row or column amax outside the
 // shortcut's range).
+// The shared tables a tile's encode reads: {value, RN(1/value)} of every
+// E4M3 code, and S_enc of the tile's 128 rows and 128 columns.
+struct EncodeTables {
+  const float2* e4m3;
+  const float* row_senc;
+  const float* col_senc;
+};
+
 template <bool kExact>
-__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm, CastStage& st,
+__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, CastStage& st,
                                              bool do_row, bool do_col, int cc, int rb,
                                              uint8_t* rdst, size_t row_pitch) {
   const int rl = 16 * rb;
@@ -179,13 +213,13 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
     }
     const uint32_t mw[4] = {m0 & 0x7FFF7FFFu, m1 & 0x7FFF7FFFu, m2 & 0x7FFF7FFFu,
                             m3 & 0x7FFF7FFFu};
-    const float* se = &sm.col_senc[8 * cc];
+    const float* se = &tab.col_senc[8 * cc];
     uint32_t s8w[2] = {0u, 0u};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
       float e0, e1;
       const uint32_t p2 = scales2_any<kExact>(bf16lo(mw[q]), se[2 * q], bf16hi(mw[q]), se[2 * q + 1],
-                                              sm.e4m3, e0, e1);
+                                              tab.e4m3, e0, e1);
       cenc2[q] = pack2(e0, e1);
       s8w[q >> 1] |= p2 << (16 * (q & 1));
     }
@@ -207,12 +241,12 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
     // the even lane of a pair scales rows 0..7, the odd lane rows 8..15
     float mine[8];
     uint32_t s8mine[2] = {0u, 0u};
-    const float* rse = &sm.row_senc[rl + (odd ? 8 : 0)];
+    const float* rse = &tab.row_senc[rl + (odd ? 8 : 0)];
 #pragma unroll
     for (int kk = 0; kk < 4; kk++) {
       const uint32_t w = odd ? P[4 + kk] : P[kk];
       const uint32_t p2 = scales2_any<kExact>(bf16lo(w), rse[2 * kk], bf16hi(w), rse[2 * kk + 1],
-                                              sm.e4m3, mine[2 * kk], mine[2 * kk + 1]);
+                                              tab.e4m3, mine[2 * kk], mine[2 * kk + 1]);
       s8mine[kk >> 1] |= p2 << (16 * (kk & 1));
     }
 #pragma unroll
@@ -279,6 +313,47 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], CastSmem& sm,
       for (int q = 0; q < 8; q++)
         *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
     }
+  }
+}
+
+// Stores of the outputs a tile staged: colwise data (64 bytes per column,
+// four 16-byte pieces), colwise scales (8 bytes per column) and rowwise scales
+// (8 bytes per row), all with the L2 evict-last policy `keep`.
+__device__ __forceinline__ void store_staged(const CastStage& st, const CastOut& out, int K,
+                                             int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
+                                             bool do_row, bool do_col, uint64_t keep) {
+  if (do_col) {
+    const size_t half_m = static_cast<size_t>(m_g) >> 1;
+    uint8_t* gd = out.col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
+#pragma unroll
+    for (int kk = 0; kk < 4; kk++) {
+      const int u = kk * kCastThreads + t;
+      const int col = u >> 2, part = u & 3;
+      const int sw = (col >> 3) & 7;
+      const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
+      const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
+      st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part,
+                        make_uint4(lo.x, lo.y, hi.x, hi.y), keep);
+    }
+    const size_t m16 = static_cast<size_t>(m_g) >> 4;
+    uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
+    uint32_t s0 = 0u, s1 = 0u;
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+      s0 |= static_cast<uint32_t>(st.col_scale[r * kCols + t]) << (8 * r);
+      s1 |= static_cast<uint32_t>(st.col_scale[(r + 4) * kCols + t]) << (8 * r);
+    }
+    st_global_u2_hint(gs + static_cast<size_t>(c0 + t) * m16, make_uint2(s0, s1), keep);
+  }
+  if (do_row) {
+    uint32_t s0 = 0u, s1 = 0u;
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+      s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
+      s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
+    }
+    st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
+                      make_uint2(s0, s1), keep);
   }
 }
 
@@ -376,13 +451,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     // this lane's 16 x 8 patch from the swizzled stage
     const bool ok = mbar_wait(&sm.full[s], phase);
     uint4 v[16];
-    {
-      const uint8_t* tb = sm.tile[s] + (cc >> 3) * kBoxBytes + rl * 128;
-      const int j = cc & 7;
-#pragma unroll
-      for (int i = 0; i < 16; i++)
-        v[i] = *reinterpret_cast<const uint4*>(tb + i * 128 + ((j ^ (i & 7)) << 4));
-    }
+    load_patch(sm.tile[s], cc, rl, v);
     if (__syncthreads_or(!ok)) {
       failed = true;
       break;
@@ -398,46 +467,14 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
 
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
                            : nullptr;
+    const EncodeTables tab{sm.e4m3, sm.row_senc, sm.col_senc};
     if (slow_tile[k & 1])
-      encode_patch<true>(v, sm, st, do_row, do_col, cc, rb, rdst, row_pitch);
+      encode_patch<true>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch);
     else
-      encode_patch<false>(v, sm, st, do_row, do_col, cc, rb, rdst, row_pitch);
+      encode_patch<false>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch);
     __syncthreads();
 
-    // ------------------------------------------------------ staged stores
-    if (do_col) {
-      const size_t half_m = static_cast<size_t>(m_g) >> 1;
-      uint8_t* gd = out.col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) {
-        const int u = kk * kCastThreads + t;
-        const int col = u >> 2, part = u & 3;
-        const int sw = (col >> 3) & 7;
-        const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
-        const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
-        st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part,
-                          make_uint4(lo.x, lo.y, hi.x, hi.y), keep);
-      }
-      const size_t m16 = static_cast<size_t>(m_g) >> 4;
-      uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
-      uint32_t s0 = 0u, s1 = 0u;
-#pragma unroll
-      for (int r = 0; r < 4; r++) {
-        s0 |= static_cast<uint32_t>(st.col_scale[r * kCols + t]) << (8 * r);
-        s1 |= static_cast<uint32_t>(st.col_scale[(r + 4) * kCols + t]) << (8 * r);
-      }
-      st_global_u2_hint(gs + static_cast<size_t>(c0 + t) * m16, make_uint2(s0, s1), keep);
-    }
-    if (do_row) {
-      uint32_t s0 = 0u, s1 = 0u;
-#pragma unroll
-      for (int r = 0; r < 4; r++) {
-        s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
-        s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
-      }
-      st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
-                        make_uint2(s0, s1), keep);
-    }
+    store_staged(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
   }
 
   if (failed && t == 0) {

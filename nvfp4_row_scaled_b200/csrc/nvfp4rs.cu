@@ -20,6 +20,7 @@
 #include "routing.cuh"
 #include "group_amax.cuh"
 #include "group_cast.cuh"
+#include "group_quantize.cuh"
 #include "dequant.cuh"
 
 using namespace nvfp4rs;
@@ -185,6 +186,72 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
                                         col_amax, o));
 }
 
+// Persistent grid of the one-launch kernel: every CTA that fits, at most one
+// per item. The schedule's lag covers the items a CTA holds at a time: one
+// per stage of its tile ring plus the next claim.
+template <class Routing>
+nvfp4_status launch_quantize(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
+                             uint32_t* ws, float* row_acc, float* row_amax, float* col_amax,
+                             const nvfp4_outputs* out, bool do_col, cudaStream_t stream) {
+  const int64_t tiles = (rows / kRows) * (K / kCols);
+  const bool s2_work = do_col && E > 0 && K > 0;
+  if (tiles == 0 && !s2_work) return NVFP4_OK;
+  CUtensorMap map;
+  if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
+  auto kernel = group_quantize_kernel<Routing>;
+  const size_t smem = quantize_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQThreads, smem) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
+  int64_t grid = static_cast<int64_t>(sms) * per_sm;
+  if (tiles > 0 && 2 * tiles < grid) grid = 2 * tiles;
+  if (grid < 1) grid = 1;
+  const int32_t lag = static_cast<int32_t>((kQStages + 1) * grid);
+  CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), lag, ws,
+                                        row_acc, row_amax, col_amax, o));
+}
+
+// Argument checks of the one-launch calls beyond check_shape / check_outputs.
+nvfp4_status check_quantize(int64_t rows, int64_t K, int32_t E, bool do_row, bool do_col,
+                            const float* row_amax, const float* col_amax, const void* workspace,
+                            size_t workspace_bytes, int64_t ws_rows) {
+  if ((do_row && rows > 0 && row_amax == nullptr) || (do_col && E > 0 && K > 0 && col_amax == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (workspace == nullptr ||
+      workspace_bytes < nvfp4_group_quantize_workspace_bytes(ws_rows, E))
+    return NVFP4_ERR_INVALID_ARG;
+  // the kernel copies 512-byte runs of both amax vectors with the TMA unit
+  if (!aligned(row_amax, 16) || !aligned(col_amax, 16) || !aligned(workspace, 16))
+    return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+// Zero what the one-launch kernel accumulates into: the workspace header, the
+// row accumulators (rows of them, when the row direction is requested) and
+// col_amax (when the column direction is).
+nvfp4_status zero_quantize_state(void* workspace, int32_t E, float* row_acc, int64_t rows, bool do_row,
+                                 float* col_amax, int64_t K, bool do_col, cudaStream_t stream) {
+  nvfp4_status s = cuda_status(cudaMemsetAsync(
+      workspace, 0, static_cast<size_t>(quant_ws_header_words(E)) * sizeof(uint32_t), stream));
+  if (s == NVFP4_OK && do_row && rows > 0)
+    s = cuda_status(cudaMemsetAsync(row_acc, 0, static_cast<size_t>(rows) * sizeof(float), stream));
+  if (s == NVFP4_OK && do_col && E > 0 && K > 0)
+    s = cuda_status(cudaMemsetAsync(col_amax, 0, static_cast<size_t>(E) * K * sizeof(float), stream));
+  return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -303,6 +370,69 @@ nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const f
   cfg.stream = stream;
   return cuda_status(cudaLaunchKernelEx(&cfg, dequant_kernel, reinterpret_cast<const uint2*>(data),
                                         scale, s2, rows, bpr, reinterpret_cast<float4*>(out_f32)));
+}
+
+size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, int32_t num_groups) {
+  if (capacity_rows < 0 || num_groups < 0 || num_groups > NVFP4_MAX_GROUPS) return 0;
+  return static_cast<size_t>(quant_ws_header_words(num_groups) + capacity_rows) * sizeof(uint32_t);
+}
+
+nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
+                                  const int64_t* m_splits_host, int32_t num_groups, float* row_amax,
+                                  float* col_amax, const nvfp4_outputs* out, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  s = check_quantize(sum_M, K, num_groups, do_row, do_col, row_amax, col_amax, workspace,
+                     workspace_bytes, 0);
+  if (s != NVFP4_OK) return s;
+  static thread_local HostRouting routing;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  if (s != NVFP4_OK) return s;
+  if (!do_row && !do_col) return NVFP4_OK;
+  // the rows accumulate straight into row_amax
+  s = zero_quantize_state(workspace, num_groups, row_amax, sum_M, do_row, col_amax, K, do_col, stream);
+  if (s != NVFP4_OK) return s;
+  return launch_quantize(routing, x_bf16, sum_M, K, num_groups, static_cast<uint32_t*>(workspace),
+                         row_amax, row_amax, col_amax, out, do_col, stream);
+}
+
+nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                            const int64_t* first_dims_dev,
+                                            const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                            float* row_amax, float* col_amax, const nvfp4_outputs* out,
+                                            void* workspace, size_t workspace_bytes,
+                                            int32_t* status_dev, cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_outputs(out, capacity_rows, K, num_groups, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  s = check_quantize(capacity_rows, K, num_groups, do_row, do_col, row_amax, col_amax, workspace,
+                     workspace_bytes, capacity_rows);
+  if (s != NVFP4_OK) return s;
+  if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
+      (num_groups > 0 && first_dims_dev == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(status_dev, 4) || !aligned(first_dims_dev, 8) || !aligned(tensor_offsets_dev, 8))
+    return NVFP4_ERR_UNSUPPORTED;
+  s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
+  if (s != NVFP4_OK || K == 0 || (!do_row && !do_col)) return s;
+  // rows beyond the routed total must stay untouched in row_amax, so the rows
+  // accumulate in the workspace and are copied out by the cast items
+  float* row_acc = reinterpret_cast<float*>(static_cast<uint32_t*>(workspace) +
+                                            quant_ws_header_words(num_groups));
+  s = zero_quantize_state(workspace, num_groups, row_acc, capacity_rows, do_row, col_amax, K, do_col,
+                          stream);
+  if (s != NVFP4_OK) return s;
+  const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
+                              num_groups};
+  return launch_quantize(routing, x_bf16, capacity_rows, K, num_groups,
+                         static_cast<uint32_t*>(workspace), row_acc, row_amax, col_amax, out, do_col,
+                         stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status status) {

@@ -90,3 +90,27 @@ def special_values_case(K=256, seed=5):
     # second group: columns of wildly different scale (colwise blocks far below the column amax)
     y = torch.randn(128, K, generator=g) * torch.exp2(torch.randint(-40, 40, (128, 1), generator=g).float())
     return torch.cat([x, y.to(torch.bfloat16)]), [128, 0, 128]
+
+
+def gpu_quantize(x: torch.Tensor, m_splits, rows=True, cols=True, device="cuda", fill=None):
+    """Host-split one-launch amax + cast on the GPU; numpy copies of all outputs.
+    ``fill`` pre-fills every output buffer with that byte (to show that every
+    byte is written)."""
+    xd = x.to(device)
+    R, K = xd.shape
+    E = len(m_splits)
+    ra, ca = abi.alloc_amax(R, K, E, device)
+    out = abi.alloc_outputs(R, K, E, device, row=rows, col=cols)
+    ws = abi.alloc_workspace(0, E, device)
+    if fill is not None:
+        for t in [ra, ca, ws, *out.values()]:
+            t.view(torch.uint8).fill_(fill)
+    abi.nvfp4_group_quantize(xd, m_splits, ra if rows else None, ca if cols else None, out, ws)
+    torch.cuda.synchronize()
+    assert int(ws[4:8].view(torch.int32).item()) == 0, "abort word raised"
+    res = {k: v.cpu().numpy() for k, v in out.items()}
+    if rows:
+        res["row_amax"] = ra.cpu().numpy()
+    if cols:
+        res["col_amax"] = ca.cpu().numpy()
+    return res

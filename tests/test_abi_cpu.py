@@ -110,6 +110,44 @@ def test_graphsafe_host_checks(L):
         abi.NVFP4_ERR_UNSUPPORTED
 
 
+def test_quantize_workspace_bytes(L):
+    f = abi.nvfp4_group_quantize_workspace_bytes
+    # 64 header words, then one done counter per group, rounded up to 64 words,
+    # then one word per row (graph-safe)
+    assert f(0, 0) == 4 * 64
+    assert f(0, 1) == 4 * 128
+    assert f(0, 64) == 4 * 128
+    assert f(0, 65) == 4 * 192
+    assert f(0, abi.NVFP4_MAX_GROUPS) == 4352
+    assert f(1000, 256) == 4 * (320 + 1000)
+    assert f(-1, 4) == 0 and f(0, -1) == 0 and f(0, abi.NVFP4_MAX_GROUPS + 1) == 0
+
+
+def test_quantize_host_checks(L):
+    arr = (ctypes.c_int64 * 2)(128, 128)
+    o = abi.Outputs(row_data=0x10000, row_scale=0x10000, row_s2=0x10000,
+                    col_data=0x10000, col_scale=0x10000, col_s2=0x10000)
+    need = abi.nvfp4_group_quantize_workspace_bytes(0, 2)
+    q = L.nvfp4_group_quantize
+
+    def call(ws=FAKE, nbytes=need, row=FAKE, col=FAKE, K=128, out=o):
+        return q(FAKE, 256, K, arr, 2, row, col, ctypes.byref(out) if out is not None else None,
+                 ws, nbytes, None)
+    assert call(ws=None) == abi.NVFP4_ERR_INVALID_ARG
+    assert call(nbytes=need - 4) == abi.NVFP4_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(0x10004)) == abi.NVFP4_ERR_UNSUPPORTED
+    assert call(row=None) == abi.NVFP4_ERR_INVALID_ARG     # rows requested, no row_amax
+    assert call(col=None) == abi.NVFP4_ERR_INVALID_ARG     # columns requested, no col_amax
+    assert call(K=120) == abi.NVFP4_ERR_INVALID_ARG
+    assert call(out=None) == abi.NVFP4_ERR_INVALID_ARG
+    g = L.nvfp4_group_quantize_graphsafe
+    small = abi.nvfp4_group_quantize_workspace_bytes(256, 2) - 4
+    assert g(FAKE, 256, 128, FAKE, FAKE, 2, FAKE, FAKE, ctypes.byref(o), FAKE, small, FAKE, None) == \
+        abi.NVFP4_ERR_INVALID_ARG  # the graph-safe call needs the row accumulators too
+    assert g(FAKE, 256, 128, FAKE, FAKE, 2, FAKE, FAKE, ctypes.byref(o), FAKE, small + 4, None, None) == \
+        abi.NVFP4_ERR_INVALID_ARG  # no status word
+
+
 def test_dequantize_host_checks(L):
     f = L.nvfp4_dequantize
     assert f(FAKE, FAKE, FAKE, 4, 24, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
