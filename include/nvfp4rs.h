@@ -238,6 +238,31 @@ NVFP4RS_API nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int6
                                             cudaStream_t stream);
 
 /*
+ * nvfp4_group_quantize without a workspace argument: the same one-launch
+ * kernel, same arguments and outputs (byte-identical), with its scratch in a
+ * static device array inside the library. This call has no counterpart in
+ * the pages the method follows. It is for callers that cannot hand over
+ * device memory at the call site: a C caller with no device allocator of
+ * its own, or one that must not allocate there (cudaMalloc synchronises the
+ * device). It allocates nothing.
+ *   - Limit: the static scratch is 4352 bytes, the workspace header of
+ *     NVFP4_MAX_GROUPS groups; larger num_groups is NVFP4_ERR_UNSUPPORTED.
+ *   - Setup: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Zeroing: each call zeroes the scratch (and row_amax, col_amax) on
+ *     `stream` before its launch; nothing needs to start at zero.
+ *   - Races: every call on a device shares the one scratch array, so calls
+ *     whose work overlaps (different streams, or threads) race and give
+ *     wrong results. Order them on one stream.
+ * row_amax and col_amax must be 16-byte aligned (else NVFP4_ERR_UNSUPPORTED).
+ */
+NVFP4RS_API nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int64_t K,
+                                          const int64_t* m_splits_host, int32_t num_groups,
+                                          float* row_amax, float* col_amax,
+                                          const nvfp4_outputs* out, cudaStream_t stream);
+
+/*
  * Dequantize one quantized matrix [rows, cols] to FP32 with one decode scale
  * per row (TransformerEngine #2931, Important Files Changed: the dequantize
  * kernel looks up the amax of the element's row, tensor_amax[y]).

@@ -71,9 +71,11 @@ def lib():
                                            vp, sz, vp]
         L.nvfp4_group_quantize_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp,
                                                      ctypes.POINTER(Outputs), vp, sz, vp, vp]
+        L.nvfp4_group_quantize_noalloc.argtypes = [vp, i64, i64, vp, i32, vp, vp,
+                                                   ctypes.POINTER(Outputs), vp]
         for f in ("nvfp4_group_amax", "nvfp4_group_cast", "nvfp4_group_amax_graphsafe",
                   "nvfp4_group_cast_graphsafe", "nvfp4_dequantize", "nvfp4_group_quantize",
-                  "nvfp4_group_quantize_graphsafe"):
+                  "nvfp4_group_quantize_graphsafe", "nvfp4_group_quantize_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         L.nvfp4_status_string.argtypes = [ctypes.c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
@@ -210,6 +212,19 @@ def nvfp4_group_quantize_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
         _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o), wp, wb,
         _dev(status, torch.int32, "status"), _stream(stream))
     _check(rc, "nvfp4_group_quantize_graphsafe")
+
+
+def nvfp4_group_quantize_noalloc(x: torch.Tensor, m_splits: Sequence[int],
+                                 row_amax: Optional[torch.Tensor], col_amax: Optional[torch.Tensor],
+                                 out: Dict[str, torch.Tensor], stream=None) -> None:
+    """nvfp4_group_quantize with the library's static scratch (no workspace)."""
+    arr, E = _splits(m_splits)
+    o = _outputs(out)
+    rc = lib().nvfp4_group_quantize_noalloc(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
+                                            _dev(row_amax, torch.float32, "row_amax"),
+                                            _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
+                                            _stream(stream))
+    _check(rc, "nvfp4_group_quantize_noalloc")
 
 
 def nvfp4_dequantize(data: torch.Tensor, scale: torch.Tensor, s2: torch.Tensor, rows: int, cols: int,

@@ -10,6 +10,7 @@
 // (TransformerEngine #3649, grouped row-scaled NVFP4 cast, Description).
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -252,6 +253,37 @@ nvfp4_status zero_quantize_state(void* workspace, int32_t E, float* row_acc, int
   return s;
 }
 
+// ------------------------------------------------ scratch without allocation
+//
+// nvfp4_group_quantize_noalloc runs the one-launch kernel with its scratch in
+// this file-scope device array instead of a caller-provided workspace. It is
+// for callers that cannot hand over device memory at the call site: a C
+// caller with no device allocator of its own, or one that must not allocate
+// there because cudaMalloc synchronises the device. The array holds the
+// workspace header for up to NVFP4_MAX_GROUPS groups (item counter, abort
+// word, one done counter per group); the row accumulators are the caller's
+// row_amax, as in the host-split call.
+constexpr int64_t kNoAllocScratchWords = quant_ws_header_words(NVFP4_MAX_GROUPS);  // 1088 words
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchWords];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch for the current device, looked up once
+// per device (with that device current) and cached. nullptr on failure.
+uint32_t* noalloc_scratch() {
+  static std::mutex mu;
+  static uint32_t* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint32_t*>(p);
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -433,6 +465,34 @@ nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity
   return launch_quantize(routing, x_bf16, capacity_rows, K, num_groups,
                          static_cast<uint32_t*>(workspace), row_acc, row_amax, col_amax, out, do_col,
                          stream);
+}
+
+nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int64_t K,
+                                          const int64_t* m_splits_host, int32_t num_groups,
+                                          float* row_amax, float* col_amax, const nvfp4_outputs* out,
+                                          cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  if ((do_row && sum_M > 0 && row_amax == nullptr) || (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(row_amax, 16) || !aligned(col_amax, 16)) return NVFP4_ERR_UNSUPPORTED;
+  // the static scratch holds the header of at most NVFP4_MAX_GROUPS groups
+  if (quant_ws_header_words(num_groups) > kNoAllocScratchWords) return NVFP4_ERR_UNSUPPORTED;
+  static thread_local HostRouting routing;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  if (s != NVFP4_OK) return s;
+  if (!do_row && !do_col) return NVFP4_OK;
+  uint32_t* scratch = noalloc_scratch();
+  if (scratch == nullptr) return NVFP4_ERR_CUDA;
+  // zeroed here on `stream`: item counter, abort word, done counters; the
+  // rows accumulate straight into row_amax, which is zeroed too
+  s = zero_quantize_state(scratch, num_groups, row_amax, sum_M, do_row, col_amax, K, do_col, stream);
+  if (s != NVFP4_OK) return s;
+  return launch_quantize(routing, x_bf16, sum_M, K, num_groups, scratch, row_amax, row_amax, col_amax, out,
+                         do_col, stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status status) {

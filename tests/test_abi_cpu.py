@@ -148,6 +148,21 @@ def test_quantize_host_checks(L):
         abi.NVFP4_ERR_INVALID_ARG  # no status word
 
 
+def test_quantize_noalloc_host_checks(L):
+    arr = (ctypes.c_int64 * 2)(128, 128)
+    o = abi.Outputs(row_data=0x10000, row_scale=0x10000, row_s2=0x10000,
+                    col_data=0x10000, col_scale=0x10000, col_s2=0x10000)
+    f = L.nvfp4_group_quantize_noalloc
+    assert f(FAKE, 256, 120, arr, 2, FAKE, FAKE, ctypes.byref(o), None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 256, 128, arr, 2, None, FAKE, ctypes.byref(o), None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 256, 128, arr, 2, ctypes.c_void_p(0x10004), FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_UNSUPPORTED  # the amax vectors are copied in 512-byte runs
+    big = (ctypes.c_int64 * (abi.NVFP4_MAX_GROUPS + 1))()
+    big[0] = 256
+    assert f(FAKE, 256, 128, big, abi.NVFP4_MAX_GROUPS + 1, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_UNSUPPORTED  # beyond the static scratch
+
+
 def test_dequantize_host_checks(L):
     f = L.nvfp4_dequantize
     assert f(FAKE, FAKE, FAKE, 4, 24, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
