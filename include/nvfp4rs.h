@@ -51,11 +51,14 @@
  *    CUDA launch returns NVFP4_ERR_CUDA. The graph-safe calls check the device
  *    routing on the device: a violation is written to *status_dev and the
  *    kernels write no output; they never trap and never hang.
- *  - Fast-path requirements (else NVFP4_ERR_UNSUPPORTED): K % 128 == 0,
- *    every group size m_g % 128 == 0 (the 128-row alignment of the grouped
- *    GEMM's scale layout), num_groups <= NVFP4_MAX_GROUPS, rows < 2^31, and
- *    every pointer 16-byte aligned. Inputs must be finite (a non-finite input
- *    gives unspecified codes, never a fault).
+ *  - Requirements (else NVFP4_ERR_UNSUPPORTED): K % 128 == 0, every group
+ *    size m_g % 16 == 0 (the colwise block height; the one-launch calls
+ *    need m_g % 128 == 0, the 128-row alignment of the grouped GEMM's scale
+ *    layout), num_groups <= NVFP4_MAX_GROUPS, rows < 2^31, and every pointer
+ *    16-byte aligned. Groups that are multiples of 128 rows take the fastest
+ *    path; others are handled per 16-row block (a 128-row tile may then hold
+ *    rows of several groups, and the last tile may be short). Inputs must be
+ *    finite (a non-finite input gives unspecified codes, never a fault).
  *  - Empty groups (m_g == 0) are allowed: their col_amax and col_s2 are 0
  *    and they own no bytes of col_data / col_scale.
  */
@@ -157,8 +160,11 @@ NVFP4RS_API nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int
  *                       offsets[num_groups] / K <= capacity_rows
  *   status_dev          device int32 [1]: set to 0 by this call, then to
  *                       NVFP4_ERR_ROUTING (inconsistent routing) or
- *                       NVFP4_ERR_UNSUPPORTED (a group not a multiple of 128
+ *                       NVFP4_ERR_UNSUPPORTED (a group not a multiple of 16
  *                       rows) by the kernel, which then writes no amax
+ * Uniform groups: with first_dims_dev and tensor_offsets_dev both NULL every
+ * group has capacity_rows / num_groups rows (which must divide exactly, else
+ * NVFP4_ERR_INVALID_ARG; a multiple of 16, else NVFP4_ERR_UNSUPPORTED).
  * One launch plus memsets of status and col_amax.
  */
 NVFP4RS_API nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
@@ -210,8 +216,10 @@ NVFP4RS_API size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, i
  *                   workspace must be ordered on one stream. After the call
  *                   word 1 is nonzero only if a bounded wait inside the kernel
  *                   gave up (not expected; the outputs are then incomplete).
- * With no direction requested nothing is enqueued. Memsets of the workspace
- * header, row_amax and col_amax, then one launch.
+ * Every group must be a multiple of 128 rows (else NVFP4_ERR_UNSUPPORTED);
+ * for other group sizes use the two calls. With no direction requested
+ * nothing is enqueued. Memsets of the workspace header, row_amax and
+ * col_amax, then one launch.
  */
 NVFP4RS_API nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
                                   const int64_t* m_splits_host, int32_t num_groups,
@@ -221,7 +229,8 @@ NVFP4RS_API nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M,
 /*
  * nvfp4_group_quantize with the graph-safe routing of
  * nvfp4_group_amax_graphsafe (same routing arguments and status rules, plus
- * NVFP4_ERR_TIMEOUT if a bounded wait gave up). Byte-identical to the
+ * NVFP4_ERR_TIMEOUT if a bounded wait gave up; a group that is not a
+ * multiple of 128 rows is NVFP4_ERR_UNSUPPORTED). Byte-identical to the
  * host-split call for equal routing, and to the graph-safe two-launch pair.
  * Rows at or beyond the routed total are neither read nor written; their row
  * amax accumulates in the workspace, which must hold

@@ -120,6 +120,16 @@ def _outputs(out: Dict[str, torch.Tensor]) -> Outputs:
     return o
 
 
+def _groups(first_dims: Optional[torch.Tensor], num_groups: Optional[int]) -> int:
+    """Group count of a graph-safe call: first_dims.numel(), or num_groups for
+    uniform groups (first_dims and tensor_offsets both None)."""
+    if first_dims is not None:
+        return first_dims.numel()
+    if num_groups is None:
+        raise ValueError("uniform groups (no first_dims) need num_groups")
+    return int(num_groups)
+
+
 def _check(rc: int, what: str):
     if rc != NVFP4_OK:
         raise NVFP4Error(what, rc)
@@ -151,11 +161,11 @@ def nvfp4_group_cast(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optiona
 def nvfp4_group_amax_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                col_amax: Optional[torch.Tensor], status: torch.Tensor,
-                               stream=None) -> None:
+                               stream=None, num_groups: Optional[int] = None) -> None:
     rc = lib().nvfp4_group_amax_graphsafe(
         _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
         _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
-        first_dims.numel(), _dev(row_amax, torch.float32, "row_amax"),
+        _groups(first_dims, num_groups), _dev(row_amax, torch.float32, "row_amax"),
         _dev(col_amax, torch.float32, "col_amax"), _dev(status, torch.int32, "status"),
         _stream(stream))
     _check(rc, "nvfp4_group_amax_graphsafe")
@@ -164,12 +174,12 @@ def nvfp4_group_amax_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
 def nvfp4_group_cast_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
-                               status: torch.Tensor, stream=None) -> None:
+                               status: torch.Tensor, stream=None, num_groups: Optional[int] = None) -> None:
     o = _outputs(out)
     rc = lib().nvfp4_group_cast_graphsafe(
         _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
         _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
-        first_dims.numel(), _dev(row_amax, torch.float32, "row_amax"),
+        _groups(first_dims, num_groups), _dev(row_amax, torch.float32, "row_amax"),
         _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
         _dev(status, torch.int32, "status"), _stream(stream))
     _check(rc, "nvfp4_group_cast_graphsafe")
@@ -202,13 +212,13 @@ def nvfp4_group_quantize_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                    tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                    col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
                                    workspace: torch.Tensor, status: torch.Tensor,
-                                   stream=None) -> None:
+                                   stream=None, num_groups: Optional[int] = None) -> None:
     o = _outputs(out)
     wp, wb = _workspace(workspace)
     rc = lib().nvfp4_group_quantize_graphsafe(
         _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
         _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
-        first_dims.numel(), _dev(row_amax, torch.float32, "row_amax"),
+        _groups(first_dims, num_groups), _dev(row_amax, torch.float32, "row_amax"),
         _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o), wp, wb,
         _dev(status, torch.int32, "status"), _stream(stream))
     _check(rc, "nvfp4_group_quantize_graphsafe")

@@ -6,8 +6,12 @@
 // is what the transposed operand is scaled by (TransformerEngine #3324,
 // summary: columnwise per-column amax).
 //
-// Work split. A 128-row tile always lies inside one group (groups are
-// multiples of 128 rows). The K/128 column chunks of a tile are dealt round
+// Work split. Tiles are 128 rows of the packed buffer; group sizes are
+// multiples of 16, so every 16-row block lies in one group. Most tiles lie
+// in one group; a "mixed" tile, which a group boundary crosses, sends each
+// lane's column maxima straight to that lane's group, and the last tile may
+// hold fewer than 128 routed rows (the rest is skipped). The K/128 column
+// chunks of a tile are dealt round
 // robin to a thread-block cluster of CN CTAs (CN <= 8, the largest divisor of
 // K/128): CTA q takes chunks q, q + CN, q + 2CN, ..., so the cluster reads each
 // row left to right in CN * 256-byte runs (much kinder to DRAM than one slab
@@ -15,8 +19,8 @@
 // quarter); warp w takes every unit of quarter w, so the four warps stay
 // balanced for any K.
 //
-// Inside a unit a lane owns 8 columns (one 16-byte chunk) of 16 rows (rows
-// 2i + h of the quarter, h = lane / 16):
+// Inside a unit a lane owns 8 columns (one 16-byte chunk) of 16 rows (the
+// 16-row block 2w + h of the tile, h = lane / 16):
 //  - column maxima: packed bf16x2 |.|-max over the lane's 16 rows, merged with
 //    the other half-warp by a shuffle, then into a per-CTA shared array;
 //  - row maxima: the lane's 8-column maximum of each of its 16 rows is
@@ -54,7 +58,7 @@ __device__ __forceinline__ void red_max_u32(float* addr, uint32_t v) {
 }
 
 template <class Routing>
-__global__ void __launch_bounds__(kAmaxThreads)
+__global__ void __launch_bounds__(kAmaxThreads, 6)
 group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restrict__ x,
                   int32_t K, int32_t cn, float* __restrict__ row_amax,
                   float* __restrict__ col_amax) {
@@ -73,6 +77,15 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   const int32_t r0 = tile * kRows;
   const int cols = K / cn;
   const bool active = rs.ok && r0 < rs.total;
+  // routed rows of the tile (a multiple of 16: the tail tile may be short),
+  // this lane's 16-row block and its group; a tile that holds rows of more
+  // than one group ("mixed") sends each lane's column maxima to its own group
+  const int valid = active ? min(kRows, rs.total - r0) : 0;
+  const int rb = 2 * warp + h;
+  const bool lane_ok = kBlockRows * rb < valid;
+  const int g_first = active ? group_of_row(rs, r0) : 0;
+  const bool mixed = active && rs.off[g_first + 1] < r0 + valid;
+  const int g_lane = (mixed && lane_ok) ? group_of_row(rs, r0 + kBlockRows * rb) : g_first;
 
   rmax[t] = 0u;
   for (int c = t; c < cols; c += kAmaxThreads) cmax[c] = 0u;
@@ -82,13 +95,15 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
     const int nchunks = cols >> 7;
     const size_t K8 = static_cast<size_t>(K) >> 3;  // row pitch in 16-byte units
     for (int ch = 0; ch < nchunks; ch++) {
-      // this lane: rows r0 + 32*warp + h + 2i (i < 16), columns c0 .. c0+7
+      // this lane: rows r0 + 16*rb + i (i < 16), columns c0 .. c0+7
       const int c_loc = (ch << 7) + (cc << 3);                // index into this CTA's cmax
       const int c_glb = ((ch * cn + rank) << 7) + (cc << 3);  // chunk ch of the CTA: rank + ch*cn
-      const uint4* p = x + (static_cast<size_t>(r0 + 32 * warp + h) * K8) + (c_glb >> 3);
+      // (a lane past the routed rows reads the tile's first block instead and
+      // contributes nothing)
+      const uint4* p = x + (static_cast<size_t>(r0 + (lane_ok ? kBlockRows * rb : 0)) * K8) + (c_glb >> 3);
       uint4 v[16];
 #pragma unroll
-      for (int i = 0; i < 16; i++) v[i] = ld_stream(p + 2 * i * K8);
+      for (int i = 0; i < 16; i++) v[i] = ld_stream(p + i * K8);
 
       // column maxima over the lane's 16 rows
       uint32_t c0 = v[0].x, c1 = v[0].y, c2 = v[0].z, c3 = v[0].w;
@@ -99,6 +114,7 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
         c2 = maxabs2(c2, v[i].z);
         c3 = maxabs2(c3, v[i].w);
       }
+      if (!lane_ok) c0 = c1 = c2 = c3 = 0u;
       // row partial maxima, packed two rows per word: P[k] = (row 2k, row 2k+1)
       uint32_t P[8];
 #pragma unroll
@@ -135,8 +151,20 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
         const uint32_t keep = b0 ? (S >> 16) : (S & 0xFFFFu);
         const uint32_t send = b0 ? (S & 0xFFFFu) : (S >> 16);
         const uint32_t rowm = max(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 1));
-        // lane (cc, h) holds local row 32*warp + h + 2*cc
-        atomicMax(&rmax[32 * warp + h + 2 * cc], rowm << 16);
+        // lane (cc, h) holds tile row 16*rb + cc
+        atomicMax(&rmax[kBlockRows * rb + cc], rowm << 16);
+      }
+      if (mixed) {  // straight to this lane's group (a mixed tile is rare)
+        if (lane_ok && col_amax != nullptr) {
+          float* dst = col_amax + static_cast<size_t>(g_lane) * K + c_glb;
+          const uint32_t w[4] = {c0 & 0x7FFF7FFFu, c1 & 0x7FFF7FFFu, c2 & 0x7FFF7FFFu, c3 & 0x7FFF7FFFu};
+#pragma unroll
+          for (int q = 0; q < 4; q++) {
+            red_max_u32(dst + 2 * q, w[q] << 16);
+            red_max_u32(dst + 2 * q + 1, w[q] & 0xFFFF0000u);
+          }
+        }
+        continue;
       }
       // merge the two half-warps' column maxima, then into the CTA's array
       c0 = maxabs2(c0, __shfl_xor_sync(0xFFFFFFFFu, c0, 16)) & 0x7FFF7FFFu;
@@ -152,15 +180,14 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
     }
   }
   __syncthreads();
-  if (active && col_amax != nullptr) {
-    const int g = group_of_row(rs, r0);
-    float* dst = col_amax + static_cast<size_t>(g) * K;
+  if (active && !mixed && col_amax != nullptr) {
+    float* dst = col_amax + static_cast<size_t>(g_first) * K;
     for (int c = t; c < cols; c += kAmaxThreads)
       red_max_u32(dst + ((((c >> 7) * cn + rank) << 7) | (c & 127)), cmax[c]);
   }
   // every CTA of the cluster reaches both barriers, active or not
   cluster.sync();
-  if (active && rank == 0 && row_amax != nullptr) {
+  if (active && rank == 0 && row_amax != nullptr && t < valid) {
     uint32_t m = rmax[t];
     for (int q = 1; q < cn; q++) m = max(m, *cluster.map_shared_rank(&rmax[t], q));
     row_amax[r0 + t] = __uint_as_float(m);

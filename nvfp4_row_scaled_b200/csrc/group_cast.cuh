@@ -11,8 +11,10 @@
 // Structure (sm_100a):
 //  - Persistent CTAs (three per SM), each taking every gridDim-th 128 x 128
 //    tile of x in row-major tile order, so CTAs running at the same time read
-//    neighbouring tiles of the same rows. A 128-row tile always lies inside
-//    one group (groups are multiples of 128 rows).
+//    neighbouring tiles of the same rows. Group sizes are multiples of 16, so
+//    a lane's 16-row block lies in one group; a tile that a group boundary
+//    crosses ("mixed") keeps one column-scale table per 16-row block, and
+//    the last tile may hold fewer than 128 routed rows.
 //  - Tiles arrive by TMA: two 2-D tiled loads of 64 columns x 128 rows each
 //    (128-byte rows, 128-byte swizzle, no multicast, L2 evict-first) into a
 //    two-stage shared-memory ring, completion tracked by one mbarrier per
@@ -31,8 +33,10 @@
 //    8-byte pieces of contiguous runs, with an L2 evict-last hint: a group's
 //    transposed outputs and the 8-byte scale pieces fill their sectors from
 //    several tiles, and should meet in L2 before being written back.
-// Every CTA also writes a slice of col_s2 = S_dec(col_amax) (all E*K
-// entries, empty groups included).
+// Tiles of groups that are not multiples of 128 rows, mixed tiles and the
+// short last tile store their colwise outputs per 16-row block
+// (store_staged_general). Every CTA also writes a slice of
+// col_s2 = S_dec(col_amax) (all E*K entries, empty groups included).
 #pragma once
 
 #include <cuda.h>
@@ -71,7 +75,7 @@ struct CastSmem {
   uint8_t tile[kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
   float2 e4m3[128];                   // {value, RN(1/value)} per E4M3 code
   float row_senc[kRows];
-  float col_senc[kCols];
+  float col_senc[kRows / kBlockRows][kCols];  // per 16-row block: [0] only, unless the tile is mixed
   uint64_t full[kStages];
 };
 
@@ -196,7 +200,7 @@ struct EncodeTables {
 template <bool kExact>
 __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, CastStage& st,
                                              bool do_row, bool do_col, int cc, int rb,
-                                             uint8_t* rdst, size_t row_pitch) {
+                                             uint8_t* rdst, size_t row_pitch, bool row_store = true) {
   const int rl = 16 * rb;
   const bool odd = cc & 1;
 
@@ -276,10 +280,12 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
                               unpack2(v[i + 1].w)};
       if (do_row) {
         const uint64_t e0 = pack2(renc[i], renc[i]), e1 = pack2(renc[i + 1], renc[i + 1]);
-        st_global_u32(rdst + i * row_pitch, e2m1_pairs(mul2x(x0[0], e0), mul2x(x0[1], e0),
-                                                       mul2x(x0[2], e0), mul2x(x0[3], e0)));
-        st_global_u32(rdst + (i + 1) * row_pitch, e2m1_pairs(mul2x(x1[0], e1), mul2x(x1[1], e1),
-                                                             mul2x(x1[2], e1), mul2x(x1[3], e1)));
+        const uint32_t w0 = e2m1_pairs(mul2x(x0[0], e0), mul2x(x0[1], e0), mul2x(x0[2], e0), mul2x(x0[3], e0));
+        const uint32_t w1 = e2m1_pairs(mul2x(x1[0], e1), mul2x(x1[1], e1), mul2x(x1[2], e1), mul2x(x1[3], e1));
+        if (row_store) {  // false for a 16-row block past the routed rows
+          st_global_u32(rdst + i * row_pitch, w0);
+          st_global_u32(rdst + (i + 1) * row_pitch, w1);
+        }
       }
       if (do_col) {
         uint64_t y0[4], y1[4];
@@ -357,9 +363,53 @@ __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut&
   }
 }
 
+// Stores of a tile that store_staged cannot take: a tile crossing a group
+// boundary, the short last tile, or a group that does not start and end on
+// 128-row boundaries (its colwise runs are then only 8-byte aligned). Colwise outputs go
+// per (column, 16-row block): 8 bytes of codes and one scale byte, to the
+// block's own group; only blocks of routed rows (16 * b < valid) are stored.
+// `g` is the tile's group when it holds one group only (mixed == false).
+__device__ __noinline__ void store_staged_general(const CastStage& st, const CastOut& out,
+                                                     const RoutingSmem& rs, int K, int32_t r0, int c0,
+                                                     int t, int valid, bool mixed, int g, bool do_row,
+                                                     bool do_col, uint64_t keep) {
+  if (do_col) {
+#pragma unroll 2
+    for (int kk = 0; kk < 8; kk++) {
+      const int u = kk * kCastThreads + t;
+      const int col = u >> 3, b = u & 7;
+      if (kBlockRows * b >= valid) continue;
+      const int32_t r = r0 + kBlockRows * b;
+      const int gb = mixed ? group_of_row(rs, r) : g;
+      const int32_t o = rs.off[gb];
+      const size_t m = static_cast<size_t>(rs.off[gb + 1] - o);
+      const int sw = (col >> 3) & 7;
+      const uint2 d = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * (b ^ sw)]);
+      st_global_u2_hint(out.col_data + (static_cast<size_t>(K) * o >> 1) + static_cast<size_t>(c0 + col) * (m >> 1) +
+                            ((r - o) >> 1),
+                        d, keep);
+      out.col_scale[(static_cast<size_t>(K) * o >> 4) + static_cast<size_t>(c0 + col) * (m >> 4) + ((r - o) >> 4)] =
+          st.col_scale[b * kCols + col];
+    }
+  }
+  if (do_row && t < valid) {
+    uint32_t s0 = 0u, s1 = 0u;
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+      s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
+      s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
+    }
+    st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
+                      make_uint2(s0, s1), keep);
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 
-template <class Routing>
+// kGeneral = false: every group is a multiple of 128 rows starting on a
+// 128-row boundary (the host checked), so every tile is plain and the
+// general-tile code is compiled out.
+template <class Routing, bool kGeneral>
 __global__ void __launch_bounds__(kCastThreads, 3)
 group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
                   int32_t K, const float* __restrict__ row_amax,
@@ -392,7 +442,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
 
   // this CTA's tiles: a contiguous range of the row-major tile order
   const int n_ct = K >> 7;
-  const int n_tiles = (rs.total >> 7) * n_ct;
+  const int n_tiles = ((rs.total + kRows - 1) >> 7) * n_ct;  // the last row tile may be short
   const int G = gridDim.x;
   if (t == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&sm.full[s], 1);
@@ -416,7 +466,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   bool failed = false;
   int cur_rt = -1;
   bool row_slow = false;
-  int g = 0;
+  int g = 0;  // group of the row tile's first row
   int32_t o_g = 0;
   int64_t m_g = 0;
   const uint64_t keep = policy_evict_last();
@@ -428,23 +478,35 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     const int c0 = ct * kCols;
     if (t == 0) slow_tile[(k + 1) & 1] = 0;  // flag of the next tile (last read a tile ago)
     bool slow = false;
-    if (rt != cur_rt) {  // new row tile: its group and its rows' encode scales
+    const int valid = kGeneral ? min(kRows, rs.total - r0) : kRows;  // routed rows (a multiple of 16)
+    if (rt != cur_rt) {  // new row tile: its group(s) and its rows' encode scales
       cur_rt = rt;
       g = group_of_row(rs, r0);
       o_g = rs.off[g];
       m_g = rs.off[g + 1] - o_g;
       if (do_row) {
-        const float a = row_amax[r0 + t];
+        const bool in = t < valid;
+        const float a = in ? row_amax[r0 + t] : 0.0f;
         sm.row_senc[t] = s_enc_of(a);
-        row_slow = !fast_path_amax(a);
-        if (ct == 0) out.row_s2[r0 + t] = s_dec_of(a);
+        row_slow = in && !fast_path_amax(a);
+        if (ct == 0 && in) out.row_s2[r0 + t] = s_dec_of(a);
       }
     }
     slow |= row_slow;
+    const bool mixed = kGeneral && o_g + m_g < r0 + valid;  // the tile crosses a group boundary
     if (do_col) {
-      const float a = col_amax[static_cast<size_t>(g) * K + c0 + t];
-      sm.col_senc[t] = s_enc_of(a);
-      slow |= !fast_path_amax(a);
+      if (!mixed) {
+        const float a = col_amax[static_cast<size_t>(g) * K + c0 + t];
+        sm.col_senc[0][t] = s_enc_of(a);
+        slow |= !fast_path_amax(a);
+      } else {  // one column table per 16-row block, from the block's group
+        for (int b = 0; kBlockRows * b < valid; b++) {
+          const int gb = group_of_row(rs, r0 + kBlockRows * b);
+          const float a = col_amax[static_cast<size_t>(gb) * K + c0 + t];
+          sm.col_senc[b][t] = s_enc_of(a);
+          slow |= !fast_path_amax(a);
+        }
+      }
     }
     if (slow) slow_tile[k & 1] = 1;
 
@@ -467,14 +529,25 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
 
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
                            : nullptr;
-    const EncodeTables tab{sm.e4m3, sm.row_senc, sm.col_senc};
+    const EncodeTables tab{sm.e4m3, sm.row_senc, sm.col_senc[mixed ? rb : 0]};
+    const bool row_store = !kGeneral || kBlockRows * rb < valid;  // false past the routed rows
     if (slow_tile[k & 1])
-      encode_patch<true>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch);
+      encode_patch<true>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
     else
-      encode_patch<false>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch);
+      encode_patch<false>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
     __syncthreads();
-
-    store_staged(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
+    // (the tile's shape again, rather than kept live through the encode) A
+    // whole tile of a group that starts and ends on 128-row boundaries takes
+    // store_staged, whose 16-byte colwise data and 8-byte colwise scale stores
+    // need those boundaries; every other tile, store_staged_general.
+    {
+      const int valid2 = kGeneral ? min(kRows, rs.total - r0) : kRows;
+      const bool mixed2 = kGeneral && o_g + m_g < r0 + valid2;
+      if (!kGeneral || (!mixed2 && valid2 == kRows && ((o_g | m_g) & (kRows - 1)) == 0))
+        store_staged(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
+      else
+        store_staged_general(st, out, rs, K, r0, c0, t, valid2, mixed2, g, do_row, do_col, keep);
+    }
   }
 
   if (failed && t == 0) {

@@ -56,8 +56,11 @@ nvfp4_status check_shape(const void* x, int64_t rows, int64_t K, int32_t E) {
   return NVFP4_OK;
 }
 
-// Host splits -> HostRouting (row offsets), with the split checks.
-nvfp4_status host_routing(const int64_t* m_splits, int32_t E, int64_t sum_M, HostRouting& r) {
+// Host splits -> HostRouting (row offsets), with the split checks. Every
+// group must be a multiple of `align` rows (16 for the two-step calls, 128
+// for the one-launch calls), else NVFP4_ERR_UNSUPPORTED.
+nvfp4_status host_routing(const int64_t* m_splits, int32_t E, int64_t sum_M, HostRouting& r,
+                          int32_t align = kBlockRows, bool* all_128 = nullptr) {
   if (E > 0 && m_splits == nullptr) return NVFP4_ERR_INVALID_ARG;
   int64_t total = 0;
   bool unaligned = false;
@@ -65,14 +68,42 @@ nvfp4_status host_routing(const int64_t* m_splits, int32_t E, int64_t sum_M, Hos
   r.off[0] = 0;
   for (int32_t g = 0; g < E; g++) {
     if (m_splits[g] < 0) return NVFP4_ERR_INVALID_ARG;
-    if (m_splits[g] % kRows != 0) unaligned = true;
+    if (m_splits[g] % align != 0) unaligned = true;
     total += m_splits[g];
     if (total > sum_M) return NVFP4_ERR_INVALID_ARG;
     r.off[g + 1] = static_cast<int32_t>(total);
   }
   if (total != sum_M) return NVFP4_ERR_INVALID_ARG;
   if (unaligned) return NVFP4_ERR_UNSUPPORTED;
+  if (all_128 != nullptr) {
+    *all_128 = true;
+    for (int32_t g = 0; g < E; g++) *all_128 = *all_128 && m_splits[g] % kRows == 0;
+  }
   r.total = static_cast<int32_t>(total);
+  return NVFP4_OK;
+}
+
+// Routing arguments of a graph-safe call -> DeviceRouting, with the host-side
+// checks. Both arrays NULL selects uniform groups: num_groups groups of
+// capacity_rows / num_groups rows each (which must divide exactly).
+nvfp4_status device_routing(const int64_t* first_dims, const int64_t* offsets, int32_t* status,
+                            int64_t K, int64_t capacity_rows, int32_t E, int32_t align,
+                            DeviceRouting& r) {
+  if (status == nullptr) return NVFP4_ERR_INVALID_ARG;
+  const bool uniform = first_dims == nullptr && offsets == nullptr;
+  int64_t m = -1;
+  if (uniform) {
+    m = 0;
+    if (E > 0) {
+      if (capacity_rows % E != 0) return NVFP4_ERR_INVALID_ARG;
+      m = capacity_rows / E;
+      if (m % align != 0) return NVFP4_ERR_UNSUPPORTED;
+    }
+  } else if (offsets == nullptr || (E > 0 && first_dims == nullptr)) {
+    return NVFP4_ERR_INVALID_ARG;
+  }
+  if (!aligned(status, 4) || !aligned(first_dims, 8) || !aligned(offsets, 8)) return NVFP4_ERR_UNSUPPORTED;
+  r = DeviceRouting{first_dims, offsets, status, K, capacity_rows, E, align, m};
   return NVFP4_OK;
 }
 
@@ -113,7 +144,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 // 128-byte swizzle (the layout the cast kernel reads back).
 bool x_tensor_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K) {
   std::memset(map, 0, sizeof(*map));
-  if (rows < kRows || K < kCols) return true;  // no full tile: the map is never used
+  if (rows == 0 || K < kCols) return true;  // no tile: the map is never used
   PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
@@ -154,16 +185,18 @@ nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t tiles, i
                                         row_amax, col_amax));
 }
 
+// general: some group may not start and end on 128-row boundaries (always
+// so for device routing, which the host cannot see).
 template <class Routing>
 nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
                          const float* row_amax, const float* col_amax, const nvfp4_outputs* out,
-                         bool do_col, cudaStream_t stream) {
-  const int64_t tiles = (rows / kRows) * (K / kCols);
+                         bool do_col, bool general, cudaStream_t stream) {
+  const int64_t tiles = ((rows + kRows - 1) / kRows) * (K / kCols);
   const bool s2_work = do_col && E > 0 && K > 0;
   if (tiles == 0 && !s2_work) return NVFP4_OK;
   CUtensorMap map;
   if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
-  auto kernel = group_cast_kernel<Routing>;
+  auto kernel = general ? group_cast_kernel<Routing, true> : group_cast_kernel<Routing, false>;
   const size_t smem = cast_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -303,7 +336,8 @@ nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
                                     stream));
     if (s != NVFP4_OK) return s;
   }
-  return launch_amax(routing, x_bf16, sum_M / kRows, K, num_groups, row_amax, col_amax, stream);
+  return launch_amax(routing, x_bf16, (sum_M + kRows - 1) / kRows, K, num_groups, row_amax, col_amax,
+                     stream);
 }
 
 nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
@@ -319,9 +353,10 @@ nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
       (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
     return NVFP4_ERR_INVALID_ARG;
   static thread_local HostRouting routing;
-  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  bool all_128 = true;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kBlockRows, &all_128);
   if (s != NVFP4_OK) return s;
-  return launch_cast(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, out, do_col,
+  return launch_cast(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, out, do_col, !all_128,
                      stream);
 }
 
@@ -332,13 +367,12 @@ nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_row
                                         cudaStream_t stream) {
   nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
   if (s != NVFP4_OK) return s;
-  if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
-      (num_groups > 0 && first_dims_dev == nullptr))
-    return NVFP4_ERR_INVALID_ARG;
+  DeviceRouting routing;
+  s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups,
+                     kBlockRows, routing);
+  if (s != NVFP4_OK) return s;
   if (capacity_rows > 0 && row_amax == nullptr && col_amax == nullptr) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(row_amax, 4) || !aligned(col_amax, 4) || !aligned(status_dev, 4) ||
-      !aligned(first_dims_dev, 8) || !aligned(tensor_offsets_dev, 8))
-    return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned(row_amax, 4) || !aligned(col_amax, 4)) return NVFP4_ERR_UNSUPPORTED;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK) return s;
   if (col_amax != nullptr && num_groups > 0 && K > 0) {
@@ -347,8 +381,6 @@ nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_row
     if (s != NVFP4_OK) return s;
   }
   if (K == 0) return NVFP4_OK;
-  const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
-                              num_groups};
   return launch_amax(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, num_groups, row_amax,
                      col_amax, stream);
 }
@@ -367,18 +399,15 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
   if ((do_row && capacity_rows > 0 && row_amax == nullptr) ||
       (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
     return NVFP4_ERR_INVALID_ARG;
-  if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
-      (num_groups > 0 && first_dims_dev == nullptr))
-    return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(status_dev, 4) || !aligned(first_dims_dev, 8) || !aligned(tensor_offsets_dev, 8))
-    return NVFP4_ERR_UNSUPPORTED;
+  DeviceRouting routing;
+  s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups,
+                     kBlockRows, routing);
+  if (s != NVFP4_OK) return s;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK) return s;
   if (K == 0) return NVFP4_OK;
-  const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
-                              num_groups};
   return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
-                     stream);
+                     /*general=*/true, stream);
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
@@ -422,7 +451,7 @@ nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
                      workspace_bytes, 0);
   if (s != NVFP4_OK) return s;
   static thread_local HostRouting routing;
-  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kRows);  // one launch: 128-row groups
   if (s != NVFP4_OK) return s;
   if (!do_row && !do_col) return NVFP4_OK;
   // the rows accumulate straight into row_amax
@@ -446,11 +475,10 @@ nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity
   s = check_quantize(capacity_rows, K, num_groups, do_row, do_col, row_amax, col_amax, workspace,
                      workspace_bytes, capacity_rows);
   if (s != NVFP4_OK) return s;
-  if (status_dev == nullptr || tensor_offsets_dev == nullptr ||
-      (num_groups > 0 && first_dims_dev == nullptr))
-    return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(status_dev, 4) || !aligned(first_dims_dev, 8) || !aligned(tensor_offsets_dev, 8))
-    return NVFP4_ERR_UNSUPPORTED;
+  DeviceRouting routing;
+  s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups, kRows,
+                     routing);
+  if (s != NVFP4_OK) return s;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK || K == 0 || (!do_row && !do_col)) return s;
   // rows beyond the routed total must stay untouched in row_amax, so the rows
@@ -460,8 +488,6 @@ nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity
   s = zero_quantize_state(workspace, num_groups, row_acc, capacity_rows, do_row, col_amax, K, do_col,
                           stream);
   if (s != NVFP4_OK) return s;
-  const DeviceRouting routing{first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows,
-                              num_groups};
   return launch_quantize(routing, x_bf16, capacity_rows, K, num_groups,
                          static_cast<uint32_t*>(workspace), row_acc, row_amax, col_amax, out, do_col,
                          stream);
@@ -482,7 +508,7 @@ nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int
   // the static scratch holds the header of at most NVFP4_MAX_GROUPS groups
   if (quant_ws_header_words(num_groups) > kNoAllocScratchWords) return NVFP4_ERR_UNSUPPORTED;
   static thread_local HostRouting routing;
-  s = host_routing(m_splits_host, num_groups, sum_M, routing);
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kRows);  // one launch: 128-row groups
   if (s != NVFP4_OK) return s;
   if (!do_row && !do_col) return NVFP4_OK;
   uint32_t* scratch = noalloc_scratch();

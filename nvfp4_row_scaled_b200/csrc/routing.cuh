@@ -22,7 +22,8 @@
 
 namespace nvfp4rs {
 
-constexpr int kRows = 128;  // rows per tile; every group is a multiple of it
+constexpr int kRows = 128;     // rows per tile
+constexpr int kBlockRows = 16; // group sizes are multiples of it: a 16-row block lies in one group
 
 // Lives in static shared memory; `off` points at E+1 int32 of dynamic shared
 // memory (sized by the host from the number of groups).
@@ -56,6 +57,9 @@ struct HostRouting {
 // Device routing: first_dims [E] rows per group, tensor_offsets [E+1]
 // element offsets (row offset * K). Checked on every load. `status` is where
 // a violation -- or a kernel's give-up on a bounded wait -- is recorded.
+// With uniform_rows >= 0 the two arrays are absent and every group has
+// uniform_rows rows (the host checked E * uniform_rows <= capacity_rows).
+// Groups whose size is not a multiple of `align` are NVFP4_ERR_UNSUPPORTED.
 struct DeviceRouting {
   const int64_t* first_dims;
   const int64_t* tensor_offsets;
@@ -63,8 +67,21 @@ struct DeviceRouting {
   int64_t K;
   int64_t capacity_rows;
   int32_t E;
+  int32_t align;
+  int64_t uniform_rows;
 
   __device__ __forceinline__ void load(RoutingSmem& s, int32_t* off_smem) const {
+    if (uniform_rows >= 0) {
+      for (int i = threadIdx.x; i <= E; i += blockDim.x) off_smem[i] = static_cast<int32_t>(i * uniform_rows);
+      if (threadIdx.x == 0) {
+        s.off = off_smem;
+        s.E = E;
+        s.ok = 1;
+        s.total = static_cast<int32_t>(E * uniform_rows);
+      }
+      __syncthreads();
+      return;
+    }
     int bad_routing = 0, bad_align = 0;
     for (int i = threadIdx.x; i <= E; i += blockDim.x) {
       const int64_t o = tensor_offsets[i];
@@ -77,7 +94,7 @@ struct DeviceRouting {
         const int64_t fd = first_dims[i];
         const int64_t next = tensor_offsets[i + 1];
         if (fd < 0 || fd > capacity_rows || next - o != fd * K) bad_routing = 1;
-        if (fd % kRows != 0) bad_align = 1;
+        if (fd % align != 0) bad_align = 1;
       }
     }
     bad_routing = __syncthreads_or(bad_routing);

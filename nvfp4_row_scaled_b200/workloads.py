@@ -130,16 +130,17 @@ def deepseek_routing(g: torch.Generator, E: int = 256, tokens: int = 8192, topk:
     return counts
 
 
-def config3(tokens: int = 8192) -> Workload:
+def config3(tokens: int = 8192, align: int = ALIGN) -> Workload:
     """DeepSeek-V3-shaped MoE input: K=7168, 256 experts, 8192 tokens top-8
     (65536 routed rows), Zipf(1.1) popularity, ~10% empty experts, every group
     padded with zero rows up to a multiple of 128; routed rows are
     N(0,1) * 2^U(-4,4) per row; seed 2. ``tokens`` scales the workload down
-    for small cases (same recipe)."""
+    for small cases (same recipe); ``align`` = 16 pads groups to multiples of
+    16 rows only (the unaligned-group variant)."""
     g = _gen(2)
     K, E = 7168, 256
     counts = deepseek_routing(g, E, tokens)
-    ms = [pad_up(c) for c in counts]
+    ms = [pad_up(c, align) for c in counts]
     rows = sum(ms)
     routed = sum(counts)
 
@@ -155,8 +156,9 @@ def config3(tokens: int = 8192) -> Workload:
         x[dst:dst + c] = dense[src:src + c]
         src += c
         dst += m
-    return Workload(f"deepseek_v3_e256_k7168_t{tokens}", K, x, ms, [],
-                    f"E=256 K=7168 {tokens} tokens top-8, Zipf(1.1), padded to 128, sum_M={rows}")
+    name = f"deepseek_v3_e256_k7168_t{tokens}" + ("" if align == ALIGN else f"_pad{align}")
+    return Workload(name, K, x, ms, [],
+                    f"E=256 K=7168 {tokens} tokens top-8, Zipf(1.1), padded to {align}, sum_M={rows}")
 
 
 def graphsafe_routing(seed: int, E: int, chunks: int, zipf: bool) -> List[int]:

@@ -72,7 +72,7 @@ def amax(L, x, sum_M, K, splits, row=FAKE, col=FAKE):
     (256, 144, [256], abi.NVFP4_ERR_UNSUPPORTED),      # K % 128 (fast path)
     (256, 128, [128, 64], abi.NVFP4_ERR_INVALID_ARG),  # splits do not add up
     (256, 128, [384, -128], abi.NVFP4_ERR_INVALID_ARG),  # negative split
-    (192, 128, [64, 128], abi.NVFP4_ERR_UNSUPPORTED),  # group not a multiple of 128
+    (192, 128, [56, 136], abi.NVFP4_ERR_UNSUPPORTED),  # group not a multiple of 16
     (-1, 128, [], abi.NVFP4_ERR_INVALID_ARG),
 ])
 def test_amax_host_checks(L, sum_M, K, splits, want):

@@ -133,9 +133,9 @@ def test_bad_device_routing_sets_status_and_writes_nothing(case):
     elif case == "negative":
         fd[0], fd[1] = -128, 384
         offs[1] = -128 * K
-    elif case == "unaligned":
-        fd[0], fd[1] = 64, 192
-        offs[1] = 64 * K
+    elif case == "unaligned":  # a group that is not a multiple of 16 rows
+        fd[0], fd[1] = 72, 184
+        offs[1] = 72 * K
         want = abi.NVFP4_ERR_UNSUPPORTED
     gs.fd.copy_(fd)
     gs.offs.copy_(offs)
