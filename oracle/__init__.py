@@ -76,6 +76,12 @@ def _declare(L):
     L.nvo_group_cast.restype = ctypes.c_int
     L.nvo_dequantize.argtypes = [_u8p, _u8p, _f32p, ctypes.c_int64, ctypes.c_int64, _f32p]
     L.nvo_dequantize.restype = ctypes.c_int
+    L.nvo_swizzle_scales_128x4.argtypes = [_u8p, ctypes.c_int64, ctypes.c_int64, _u8p]
+    L.nvo_swizzle_scales_128x4.restype = ctypes.c_int
+    L.nvo_f32_to_bf16.argtypes = [ctypes.c_float]
+    L.nvo_f32_to_bf16.restype = ctypes.c_uint16
+    L.nvo_row_post_scale.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int64, _f32p, _f32p, _f32p, _u16p]
+    L.nvo_row_post_scale.restype = ctypes.c_int
 
 
 class OracleError(RuntimeError):
@@ -221,3 +227,52 @@ def col_slice(col_flat: np.ndarray, m_splits: Sequence[int], K: int, g: int, per
     m = ms[g]
     start = K * o // per_elem
     return col_flat[start:start + K * m // per_elem].reshape(K, m // per_elem)
+
+
+# --------------------------------------------------- consumer side of the cast
+
+def swizzle_scales_128x4(scale: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """The 128x4-tiled layout of a scale matrix [rows, cols] (flat uint8,
+    ceil(rows/128)*128 * ceil(cols/4)*4 bytes)."""
+    scale = np.ascontiguousarray(scale, dtype=np.uint8).reshape(-1)
+    assert scale.size == rows * cols
+    out = np.zeros(((rows + 127) // 128) * 128 * ((cols + 3) // 4) * 4, dtype=np.uint8)
+    _check(lib().nvo_swizzle_scales_128x4(_ptr(scale, _u8p), rows, cols, _ptr(out, _u8p)),
+           "swizzle_scales_128x4")
+    return out
+
+
+def f32_to_bf16(v: float) -> int:
+    return int(lib().nvo_f32_to_bf16(float(v)))
+
+
+def row_post_scale(x: np.ndarray, amax: np.ndarray, bias: Optional[np.ndarray] = None):
+    """(f32 [rows, cols], bf16 bits [rows, cols]) of the per-row post-scale."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    amax = np.ascontiguousarray(amax, dtype=np.float32).reshape(-1)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32).reshape(-1)
+    of = np.zeros((rows, cols), dtype=np.float32)
+    ob = np.zeros((rows, cols), dtype=np.uint16)
+    _check(lib().nvo_row_post_scale(_ptr(x, _f32p), rows, cols, _ptr(amax, _f32p), _ptr(b, _f32p),
+                                    _ptr(of, _f32p), _ptr(ob, _u16p)), "row_post_scale")
+    return of, ob
+
+
+def swizzle_cast_scales(out: dict, m_splits: Sequence[int], K: int) -> dict:
+    """The scale outputs of a grouped cast in the 128x4-tiled layout: rowwise
+    [sum_M, K/16] as one matrix, colwise per group [K, m_g/16] at its own
+    offset K*o_g/16 (groups must be multiples of 128 rows)."""
+    res = {}
+    if "row_scale" in out:
+        rs = np.asarray(out["row_scale"]).reshape(-1)
+        rows = rs.size // (K // 16)
+        res["row_scale"] = swizzle_scales_128x4(rs, rows, K // 16)
+    if "col_scale" in out:
+        cs = np.asarray(out["col_scale"]).reshape(-1)
+        parts = []
+        for g, m in enumerate(m_splits):
+            if m:
+                parts.append(swizzle_scales_128x4(col_slice(cs, m_splits, K, g, 16), K, m // 16))
+        res["col_scale"] = np.concatenate(parts) if parts else np.zeros(0, np.uint8)
+    return res

@@ -290,6 +290,52 @@ int nvo_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
   return NVO_OK;
 }
 
+/* ------------------------------------------------ consumer side of the cast */
+
+/* [T] the 128x4-tiled scale layout, written straight from its index map */
+int nvo_swizzle_scales_128x4(const uint8_t* scale, int64_t rows, int64_t cols, uint8_t* out) {
+  if (rows < 0 || cols < 0) return NVO_E_ARG;
+  const int64_t row_tiles = (rows + 127) / 128, col_tiles = (cols + 3) / 4;
+  if (row_tiles * col_tiles > 0 && out == NULL) return NVO_E_ARG;
+  if (rows * cols > 0 && scale == NULL) return NVO_E_ARG;
+  for (int64_t i = 0; i < row_tiles * col_tiles * 512; i++) out[i] = 0;
+  for (int64_t r = 0; r < rows; r++) {
+    for (int64_t c = 0; c < cols; c++) {
+      const int64_t tile = (r / 128) * col_tiles + (c / 4);
+      const int64_t rr = r % 128, cc = c % 4;
+      out[tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + cc] = scale[r * cols + c];
+    }
+  }
+  return NVO_OK;
+}
+
+/* [T] round to nearest even on the 16 bits that are dropped: add half an
+ * ulp of the result, less one unless the kept part is odd, and truncate */
+uint16_t nvo_f32_to_bf16(float v) {
+  uint32_t b;
+  memcpy(&b, &v, sizeof b);
+  if ((b & 0x7F800000u) == 0x7F800000u && (b & 0x007FFFFFu) != 0u)
+    return (uint16_t)((b >> 16) | 0x0040u); /* NaN: keep it a (quiet) NaN */
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return (uint16_t)(b >> 16);
+}
+
+/* [T] post-GEMM row scaling, one rounding per operation */
+int nvo_row_post_scale(const float* in, int64_t rows, int64_t cols, const float* amax,
+                       const float* bias, float* out_f32, uint16_t* out_bf16) {
+  if (rows < 0 || cols < 0) return NVO_E_ARG;
+  if (rows * cols > 0 && (in == NULL || amax == NULL)) return NVO_E_ARG;
+  for (int64_t r = 0; r < rows; r++) {
+    for (int64_t c = 0; c < cols; c++) {
+      float y = in[r * cols + c] * amax[r];
+      if (bias != NULL) y = y + bias[c];
+      if (out_f32 != NULL) out_f32[r * cols + c] = y;
+      if (out_bf16 != NULL) out_bf16[r * cols + c] = nvo_f32_to_bf16(y);
+    }
+  }
+  return NVO_OK;
+}
+
 /* --------------------------------------------- array forms for the tests */
 
 void nvo_e2m1_encode_array(const float* y, int64_t n, uint8_t* out) {

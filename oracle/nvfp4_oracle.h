@@ -77,6 +77,32 @@ int nvo_group_cast(const uint16_t* x, int64_t sum_M, int64_t K,
 int nvo_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
                    int64_t rows, int64_t cols, float* out);
 
+/* ------------------------------------------------ consumer side of the cast */
+
+/* The 128x4-tiled scale layout that block-scaled grouped GEMMs read (the
+ * "swizzle contract" of "[NVFP4 4over6] Add the grouped-experts four-over-six
+ * converter" (torchtitan #14), Design notes, which needs 128-row-aligned
+ * token groups; TransformerEngine #3649's review asks the same alignment of
+ * uniform expert sizes). The pages do not print the layout. Reading: the
+ * scale matrix [rows, cols] is
+ * cut into tiles of 128 rows x 4 columns (zero padded at the edges), stored
+ * one after another in row-major tile order, 512 bytes each; inside a tile,
+ * element (r, c) sits at byte (r % 32) * 16 + (r / 32) * 4 + c. out holds
+ * ceil(rows/128)*128 * ceil(cols/4)*4 bytes. */
+int nvo_swizzle_scales_128x4(const uint8_t* scale, int64_t rows, int64_t cols, uint8_t* out);
+
+/* IEEE binary32 -> bfloat16 bits, round to nearest even (NaN stays NaN). */
+uint16_t nvo_f32_to_bf16(float v);
+
+/* The FP32 post-scale after a GEMM run with the row amax replaced by ones
+ * (TransformerEngine #2931, sequence diagram: the output rows are multiplied
+ * by the row-wise scales, then converted to the target dtype; the bias is
+ * taken out before and added back after). y[r][c] = fl(in[r][c] * amax[r]),
+ * then, with a bias, fl(y + bias[c]). out_f32 and out_bf16 (RNE of y) may
+ * each be NULL; bias may be NULL. */
+int nvo_row_post_scale(const float* in, int64_t rows, int64_t cols, const float* amax,
+                       const float* bias, float* out_f32, uint16_t* out_bf16);
+
 #ifdef __cplusplus
 }
 #endif
