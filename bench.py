@@ -307,6 +307,43 @@ def main():
     barrier()
     one_ms = max_over_ranks(q0.elapsed_time(q1) / args.steps, world, dev)
 
+    # ---- consumer side: the same step with both scale outputs in the
+    # 128x4-tiled layout, and the post-GEMM row scaling of an fp32 GEMM
+    # output [sum_M, 2048] (+ bias) to bf16
+    def timed(fn, n):
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n):
+            fn()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        return a0.elapsed_time(a1) / n
+
+    def tiled_step():
+        abi.nvfp4_group_amax(x, splits, ra, ca)
+        abi.nvfp4_group_cast(x, splits, ra, ca, out, scale_layout=abi.NVFP4_SCALE_TILED_128X4)
+
+    for _ in range(args.warmup):
+        tiled_step()
+    barrier()
+    tiled_ms = max_over_ranks(timed(tiled_step, args.steps), world, dev)
+    step()  # leave the compact outputs for the end-to-end leg
+    POST_N = 2048
+    gemm_out = torch.randn(M, POST_N, device=dev)
+    post_out = torch.empty(M, POST_N, dtype=torch.bfloat16, device=dev)
+    post_bias = torch.randn(POST_N, device=dev)
+
+    def post():
+        abi.nvfp4_row_post_scale(gemm_out, ra, post_out, post_bias)
+
+    for _ in range(args.warmup):
+        post()
+    barrier()
+    post_ms = max_over_ranks(timed(post, args.steps), world, dev)
+    post_bytes = M * POST_N * (4 + 2) + 4 * M + 4 * POST_N
+    del gemm_out, post_out
+
     # ---- end to end through the C ABI with host buffers (pinned)
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
     e2e_steps = max(3, min(args.steps, 5))
@@ -396,6 +433,16 @@ def main():
             "hbm_gbs": round(b["cast"] / (one_ms * 1e-3) / 1e9, 1),
             "hbm_frac_of_peak": round(b["cast"] / (one_ms * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes_per_launch": b["cast"],
+        },
+        "consumer": {
+            "tiled_scales_ms_per_step": round(tiled_ms, 4),
+            "tiled_scales_value": round(job_throughput(N, world, tiled_ms), 3),
+            "post_scale": {
+                "shape": [M, POST_N], "out": "bf16", "bias": True,
+                "ms": round(post_ms, 4),
+                "hbm_gbs": round(post_bytes / (post_ms * 1e-3) / 1e9, 1),
+                "hbm_frac_of_peak": round(post_bytes / (post_ms * 1e-3) / 1e9 / peak, 4),
+            },
         },
         "gpu_launches": 2 * args.steps,
         "clocks": clk,

@@ -95,6 +95,18 @@ typedef enum {
 #define NVFP4RS_API
 #endif
 
+/* Layout of the E4M3 block-scale outputs. */
+typedef enum {
+  NVFP4_SCALE_COMPACT = 0,   /* row-major [rows, cols] as listed above */
+  NVFP4_SCALE_TILED_128X4 = 1 /* the 128x4-tiled layout block-scaled GEMMs read: the
+                                 matrix [rows, cols] in tiles of 128 rows x 4 columns,
+                                 512 bytes each, in row-major tile order; scale (r, c) of
+                                 a tile at byte (r % 32) * 16 + (r / 32) * 4 + c. Same
+                                 sizes and per-group offsets as compact. Needs every
+                                 group to be a multiple of 128 rows (else
+                                 NVFP4_ERR_UNSUPPORTED). */
+} nvfp4_scale_layout;
+
 /* Output buffers of the grouped cast (device pointers). A direction whose
  * three pointers are all NULL is skipped; a direction with some but not all
  * three set is NVFP4_ERR_INVALID_ARG. */
@@ -105,6 +117,7 @@ typedef struct {
   uint8_t* col_data;  /* per group [K, m_g/2] at byte K*o_g/2   */
   uint8_t* col_scale; /* per group [K, m_g/16] at byte K*o_g/16 */
   float* col_s2;      /* [E*K]         */
+  int32_t scale_layout; /* nvfp4_scale_layout of row_scale and col_scale (0 = compact) */
 } nvfp4_outputs;
 
 /*
@@ -285,6 +298,30 @@ NVFP4RS_API nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_
  */
 NVFP4RS_API nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
                               int64_t rows, int64_t cols, float* out_f32, cudaStream_t stream);
+
+/* Output type of nvfp4_row_post_scale. */
+typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
+
+/*
+ * Per-row FP32 scaling of a GEMM output (TransformerEngine #2931, sequence
+ * diagram: the GEMM runs with the row-scaled operand's amax replaced by
+ * ones, then its output rows are multiplied by the row-wise amax and
+ * converted to the target dtype; gemm.py in Important Files Changed: the
+ * bias is taken out before and added back after). For every element
+ *   y = fl(gemm_out[r][c] * row_amax[r]);  with a bias y = fl(y + bias[c]);
+ *   out[r][c] = y as f32, or as bf16 (round to nearest even).
+ *   gemm_out   device fp32 [rows, cols], row-major
+ *   row_amax   device fp32 [rows] (the row amax of the row-scaled operand,
+ *              e.g. row_amax of the grouped amax for packed expert rows)
+ *   bias       device fp32 [cols], or NULL
+ *   out        device [rows, cols] of out_dtype; may be gemm_out itself
+ *              for NVFP4_OUT_F32 (in place)
+ * Requires cols % 4 == 0, gemm_out and bias 16-byte aligned, out 16-byte
+ * (f32) or 8-byte (bf16) aligned (else NVFP4_ERR_UNSUPPORTED). One launch.
+ */
+NVFP4RS_API nvfp4_status nvfp4_row_post_scale(const float* gemm_out, int64_t rows, int64_t cols,
+                                  const float* row_amax, const float* bias, void* out,
+                                  int32_t out_dtype, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 NVFP4RS_API const char* nvfp4_status_string(nvfp4_status status);

@@ -32,6 +32,10 @@ NVFP4_ERR_CUDA = 3
 NVFP4_ERR_ROUTING = 4
 NVFP4_ERR_TIMEOUT = 5
 NVFP4_MAX_GROUPS = 1024
+NVFP4_SCALE_COMPACT = 0
+NVFP4_SCALE_TILED_128X4 = 1
+NVFP4_OUT_F32 = 0
+NVFP4_OUT_BF16 = 1
 
 _lib = None
 
@@ -46,7 +50,8 @@ class Outputs(ctypes.Structure):
     """Mirror of ``nvfp4_outputs``."""
     _fields_ = [("row_data", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
                 ("row_s2", ctypes.c_void_p), ("col_data", ctypes.c_void_p),
-                ("col_scale", ctypes.c_void_p), ("col_s2", ctypes.c_void_p)]
+                ("col_scale", ctypes.c_void_p), ("col_s2", ctypes.c_void_p),
+                ("scale_layout", ctypes.c_int32)]
 
 
 def lib():
@@ -71,6 +76,8 @@ def lib():
                                            vp, sz, vp]
         L.nvfp4_group_quantize_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp,
                                                      ctypes.POINTER(Outputs), vp, sz, vp, vp]
+        L.nvfp4_row_post_scale.argtypes = [vp, i64, i64, vp, vp, vp, i32, vp]
+        L.nvfp4_row_post_scale.restype = ctypes.c_int
         L.nvfp4_group_quantize_noalloc.argtypes = [vp, i64, i64, vp, i32, vp, vp,
                                                    ctypes.POINTER(Outputs), vp]
         for f in ("nvfp4_group_amax", "nvfp4_group_cast", "nvfp4_group_amax_graphsafe",
@@ -111,8 +118,9 @@ def _splits(m_splits: Sequence[int]):
     return arr, len(m_splits)
 
 
-def _outputs(out: Dict[str, torch.Tensor]) -> Outputs:
+def _outputs(out: Dict[str, torch.Tensor], scale_layout: int = NVFP4_SCALE_COMPACT) -> Outputs:
     o = Outputs()
+    o.scale_layout = int(scale_layout)
     for name, dt in (("row_data", torch.uint8), ("row_scale", torch.uint8), ("row_s2", torch.float32),
                      ("col_data", torch.uint8), ("col_scale", torch.uint8), ("col_s2", torch.float32)):
         p = _dev(out.get(name), dt, name)
@@ -148,9 +156,9 @@ def nvfp4_group_amax(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optiona
 
 def nvfp4_group_cast(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optional[torch.Tensor],
                      col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
-                     stream=None) -> None:
+                     stream=None, scale_layout: int = NVFP4_SCALE_COMPACT) -> None:
     arr, E = _splits(m_splits)
-    o = _outputs(out)
+    o = _outputs(out, scale_layout)
     rc = lib().nvfp4_group_cast(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
                                 _dev(row_amax, torch.float32, "row_amax"),
                                 _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
@@ -174,8 +182,8 @@ def nvfp4_group_amax_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
 def nvfp4_group_cast_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
-                               status: torch.Tensor, stream=None, num_groups: Optional[int] = None) -> None:
-    o = _outputs(out)
+                               status: torch.Tensor, stream=None, scale_layout: int = NVFP4_SCALE_COMPACT, num_groups: Optional[int] = None) -> None:
+    o = _outputs(out, scale_layout)
     rc = lib().nvfp4_group_cast_graphsafe(
         _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
         _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
@@ -197,9 +205,9 @@ def _workspace(ws: torch.Tensor):
 
 def nvfp4_group_quantize(x: torch.Tensor, m_splits: Sequence[int], row_amax: Optional[torch.Tensor],
                          col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
-                         workspace: torch.Tensor, stream=None) -> None:
+                         workspace: torch.Tensor, stream=None, scale_layout: int = NVFP4_SCALE_COMPACT) -> None:
     arr, E = _splits(m_splits)
-    o = _outputs(out)
+    o = _outputs(out, scale_layout)
     wp, wb = _workspace(workspace)
     rc = lib().nvfp4_group_quantize(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
                                     _dev(row_amax, torch.float32, "row_amax"),
@@ -212,8 +220,8 @@ def nvfp4_group_quantize_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                    tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                    col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
                                    workspace: torch.Tensor, status: torch.Tensor,
-                                   stream=None, num_groups: Optional[int] = None) -> None:
-    o = _outputs(out)
+                                   stream=None, scale_layout: int = NVFP4_SCALE_COMPACT, num_groups: Optional[int] = None) -> None:
+    o = _outputs(out, scale_layout)
     wp, wb = _workspace(workspace)
     rc = lib().nvfp4_group_quantize_graphsafe(
         _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
@@ -226,15 +234,34 @@ def nvfp4_group_quantize_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
 
 def nvfp4_group_quantize_noalloc(x: torch.Tensor, m_splits: Sequence[int],
                                  row_amax: Optional[torch.Tensor], col_amax: Optional[torch.Tensor],
-                                 out: Dict[str, torch.Tensor], stream=None) -> None:
+                                 out: Dict[str, torch.Tensor], stream=None, scale_layout: int = NVFP4_SCALE_COMPACT) -> None:
     """nvfp4_group_quantize with the library's static scratch (no workspace)."""
     arr, E = _splits(m_splits)
-    o = _outputs(out)
+    o = _outputs(out, scale_layout)
     rc = lib().nvfp4_group_quantize_noalloc(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
                                             _dev(row_amax, torch.float32, "row_amax"),
                                             _dev(col_amax, torch.float32, "col_amax"), ctypes.byref(o),
                                             _stream(stream))
     _check(rc, "nvfp4_group_quantize_noalloc")
+
+
+def nvfp4_row_post_scale(gemm_out: torch.Tensor, row_amax: torch.Tensor, out: torch.Tensor,
+                         bias: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out = gemm_out * row_amax[:, None] (+ bias), as fp32 or bf16 (out's dtype)."""
+    if out.dtype == torch.float32:
+        dt = NVFP4_OUT_F32
+    elif out.dtype == torch.bfloat16:
+        dt = NVFP4_OUT_BF16
+    else:
+        raise ValueError("out must be float32 or bfloat16")
+    if out.shape != gemm_out.shape:
+        raise ValueError("out must have gemm_out's shape")
+    rows, cols = gemm_out.shape
+    rc = lib().nvfp4_row_post_scale(_dev(gemm_out, torch.float32, "gemm_out"), rows, cols,
+                                    _dev(row_amax, torch.float32, "row_amax"),
+                                    _dev(bias, torch.float32, "bias"), _dev(out, out.dtype, "out"), dt,
+                                    _stream(stream))
+    _check(rc, "nvfp4_row_post_scale")
 
 
 def nvfp4_dequantize(data: torch.Tensor, scale: torch.Tensor, s2: torch.Tensor, rows: int, cols: int,

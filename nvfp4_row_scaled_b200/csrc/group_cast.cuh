@@ -61,6 +61,7 @@ struct CastOut {
   uint8_t* col_data;
   uint8_t* col_scale;
   float* col_s2;
+  int32_t tiled_scales;  // nonzero: both scale outputs in the 128x4-tiled layout
 };
 
 // Output staging of one tile.
@@ -322,9 +323,30 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
   }
 }
 
+// The 128x4-tiled scale layout (the grouped GEMM's swizzle contract; see the
+// oracle for the reading): in a 512-byte tile, scale (r, c) sits at byte
+// (r % 32) * 16 + (r / 32) * 4 + c. A tile of this kernel fills two such
+// tiles; thread t (of 128) writes 8 bytes of tile t / 64: rows q, q + 32 (t
+// even) or q + 64, q + 96 (t odd) with q = (t / 2) % 32, columns 0..3 each,
+// taken from staged scales stg[c * 128 + r] (c = 16-element block 0..3).
+__device__ __forceinline__ uint32_t tiled_piece_offset(int t) { return 16u * ((t >> 1) & 31) + 8u * (t & 1); }
+
+__device__ __forceinline__ uint2 tiled_piece(const uint8_t* stg, int t) {
+  const int q = (t >> 1) & 31, i0 = 2 * (t & 1);
+  uint32_t w[2];
+#pragma unroll
+  for (int ii = 0; ii < 2; ii++) {
+    const int r = q + 32 * (i0 + ii);
+    w[ii] = static_cast<uint32_t>(stg[r]) | (static_cast<uint32_t>(stg[kRows + r]) << 8) |
+            (static_cast<uint32_t>(stg[2 * kRows + r]) << 16) | (static_cast<uint32_t>(stg[3 * kRows + r]) << 24);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
 // Stores of the outputs a tile staged: colwise data (64 bytes per column,
 // four 16-byte pieces), colwise scales (8 bytes per column) and rowwise scales
 // (8 bytes per row), all with the L2 evict-last policy `keep`.
+template <bool kTiled>
 __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut& out, int K,
                                              int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
                                              bool do_row, bool do_col, uint64_t keep) {
@@ -341,29 +363,48 @@ __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut&
       st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part,
                         make_uint4(lo.x, lo.y, hi.x, hi.y), keep);
     }
-    const size_t m16 = static_cast<size_t>(m_g) >> 4;
-    uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
-    uint32_t s0 = 0u, s1 = 0u;
+    if (kTiled) {
+      // the tile's 128 x 8 block scales are two whole 128x4 tiles of the
+      // group's [K, m_g/16] scale matrix: tile row c0/128, tile columns
+      // (r0 - o_g)/64 + 0, 1 (m_g/64 tiles per tile row)
+      const int j = t >> 6;
+      uint8_t* blk = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) +
+                     ((static_cast<size_t>(c0 >> 7) * (static_cast<size_t>(m_g) >> 6)) + ((r0 - o_g) >> 6) + j) * 512;
+      st_global_u2_hint(blk + tiled_piece_offset(t), tiled_piece(st.col_scale + 4 * j * kCols, t), keep);
+    } else {
+      const size_t m16 = static_cast<size_t>(m_g) >> 4;
+      uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
+      uint32_t s0 = 0u, s1 = 0u;
 #pragma unroll
-    for (int r = 0; r < 4; r++) {
-      s0 |= static_cast<uint32_t>(st.col_scale[r * kCols + t]) << (8 * r);
-      s1 |= static_cast<uint32_t>(st.col_scale[(r + 4) * kCols + t]) << (8 * r);
+      for (int r = 0; r < 4; r++) {
+        s0 |= static_cast<uint32_t>(st.col_scale[r * kCols + t]) << (8 * r);
+        s1 |= static_cast<uint32_t>(st.col_scale[(r + 4) * kCols + t]) << (8 * r);
+      }
+      st_global_u2_hint(gs + static_cast<size_t>(c0 + t) * m16, make_uint2(s0, s1), keep);
     }
-    st_global_u2_hint(gs + static_cast<size_t>(c0 + t) * m16, make_uint2(s0, s1), keep);
   }
   if (do_row) {
-    uint32_t s0 = 0u, s1 = 0u;
+    if (kTiled) {
+      // two whole 128x4 tiles of the [rows, K/16] scale matrix: tile row
+      // r0/128, tile columns c0/64 + 0, 1 (K/64 tiles per tile row)
+      const int j = t >> 6;
+      uint8_t* blk = out.row_scale + (static_cast<size_t>(r0 >> 7) * (K >> 6) + (c0 >> 6) + j) * 512;
+      st_global_u2_hint(blk + tiled_piece_offset(t), tiled_piece(st.row_scale + 4 * j * kRows, t), keep);
+    } else {
+      uint32_t s0 = 0u, s1 = 0u;
 #pragma unroll
-    for (int r = 0; r < 4; r++) {
-      s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
-      s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
+      for (int r = 0; r < 4; r++) {
+        s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
+        s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
+      }
+      st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
+                        make_uint2(s0, s1), keep);
     }
-    st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
-                      make_uint2(s0, s1), keep);
   }
 }
 
-// Stores of a tile that store_staged cannot take: a tile crossing a group
+// (Never sees tiled scales: those need 128-aligned groups, whose tiles are
+// all plain.) Stores of a tile that store_staged cannot take: a tile crossing a group
 // boundary, the short last tile, or a group that does not start and end on
 // 128-row boundaries (its colwise runs are then only 8-byte aligned). Colwise outputs go
 // per (column, 16-row block): 8 bytes of codes and one scale byte, to the
@@ -407,9 +448,10 @@ __device__ __noinline__ void store_staged_general(const CastStage& st, const Cas
 // ------------------------------------------------------------------ kernel
 
 // kGeneral = false: every group is a multiple of 128 rows starting on a
-// 128-row boundary (the host checked), so every tile is plain and the
-// general-tile code is compiled out.
-template <class Routing, bool kGeneral>
+// 128-row boundary (the host or the device routing checked), so every tile
+// is plain and the general-tile code is compiled out. kTiled: both scale
+// outputs in the 128x4-tiled layout (only with kGeneral = false).
+template <class Routing, bool kGeneral, bool kTiled>
 __global__ void __launch_bounds__(kCastThreads, 3)
 group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
                   int32_t K, const float* __restrict__ row_amax,
@@ -544,7 +586,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
       const int valid2 = kGeneral ? min(kRows, rs.total - r0) : kRows;
       const bool mixed2 = kGeneral && o_g + m_g < r0 + valid2;
       if (!kGeneral || (!mixed2 && valid2 == kRows && ((o_g | m_g) & (kRows - 1)) == 0))
-        store_staged(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
+        store_staged<kTiled>(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
       else
         store_staged_general(st, out, rs, K, r0, c0, t, valid2, mixed2, g, do_row, do_col, keep);
     }

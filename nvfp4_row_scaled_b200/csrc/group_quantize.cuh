@@ -220,7 +220,8 @@ __device__ __forceinline__ bool wait_group(const uint32_t* done, uint32_t need, 
 
 // ----------------------------------------------------------------- kernel
 
-template <class Routing>
+// kTiled: both scale outputs in the 128x4-tiled layout.
+template <class Routing, bool kTiled>
 __global__ void __launch_bounds__(kQThreads, 2)
 group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
                       int32_t K, int32_t lag, uint32_t* ws, float* row_acc, float* row_amax,
@@ -492,7 +493,7 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
       else
         encode_patch<false>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch);
       compute_bar();
-      store_staged(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
+      store_staged<kTiled>(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
     }
     // this thread's generic writes to the stage come before the next TMA load into it
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -23,6 +23,7 @@
 #include "group_cast.cuh"
 #include "group_quantize.cuh"
 #include "dequant.cuh"
+#include "post_scale.cuh"
 
 using namespace nvfp4rs;
 
@@ -113,6 +114,8 @@ nvfp4_status device_routing(const int64_t* first_dims, const int64_t* offsets, i
 nvfp4_status check_outputs(const nvfp4_outputs* out, int64_t rows, int64_t K, int32_t E,
                            bool& do_row, bool& do_col) {
   if (out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (out->scale_layout != NVFP4_SCALE_COMPACT && out->scale_layout != NVFP4_SCALE_TILED_128X4)
+    return NVFP4_ERR_INVALID_ARG;
   do_row = out->row_data != nullptr || out->row_scale != nullptr || out->row_s2 != nullptr;
   do_col = out->col_data != nullptr || out->col_scale != nullptr || out->col_s2 != nullptr;
   const bool has_rows = rows > 0 && K > 0;
@@ -196,7 +199,11 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
   if (tiles == 0 && !s2_work) return NVFP4_OK;
   CUtensorMap map;
   if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
-  auto kernel = general ? group_cast_kernel<Routing, true> : group_cast_kernel<Routing, false>;
+  // tiled scales come with 128-row groups only (checked on the host, or on
+  // the device by the routing), so their tiles are all plain
+  const bool tiled = out->scale_layout == NVFP4_SCALE_TILED_128X4;
+  auto kernel = tiled ? group_cast_kernel<Routing, false, true>
+                      : (general ? group_cast_kernel<Routing, true, false> : group_cast_kernel<Routing, false, false>);
   const size_t smem = cast_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -210,7 +217,8 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
   if (tiles > 0 && tiles < grid) grid = tiles;
   if (grid < 1) grid = 1;
-  CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2};
+  CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2,
+            out->scale_layout == NVFP4_SCALE_TILED_128X4};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kCastThreads);
@@ -232,7 +240,8 @@ nvfp4_status launch_quantize(const Routing& routing, const void* x, int64_t rows
   if (tiles == 0 && !s2_work) return NVFP4_OK;
   CUtensorMap map;
   if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
-  auto kernel = group_quantize_kernel<Routing>;
+  auto kernel = out->scale_layout == NVFP4_SCALE_TILED_128X4 ? group_quantize_kernel<Routing, true>
+                                                             : group_quantize_kernel<Routing, false>;
   const size_t smem = quantize_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -247,7 +256,8 @@ nvfp4_status launch_quantize(const Routing& routing, const void* x, int64_t rows
   if (tiles > 0 && 2 * tiles < grid) grid = 2 * tiles;
   if (grid < 1) grid = 1;
   const int32_t lag = static_cast<int32_t>((kQStages + 1) * grid);
-  CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2};
+  CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2,
+            out->scale_layout == NVFP4_SCALE_TILED_128X4};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kQThreads);
@@ -356,6 +366,7 @@ nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
   bool all_128 = true;
   s = host_routing(m_splits_host, num_groups, sum_M, routing, kBlockRows, &all_128);
   if (s != NVFP4_OK) return s;
+  if (out->scale_layout == NVFP4_SCALE_TILED_128X4 && !all_128) return NVFP4_ERR_UNSUPPORTED;
   return launch_cast(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, out, do_col, !all_128,
                      stream);
 }
@@ -399,9 +410,9 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
   if ((do_row && capacity_rows > 0 && row_amax == nullptr) ||
       (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
     return NVFP4_ERR_INVALID_ARG;
-  DeviceRouting routing;
+  DeviceRouting routing;  // tiled scales need 128-row groups: checked on the device
   s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups,
-                     kBlockRows, routing);
+                     out->scale_layout == NVFP4_SCALE_TILED_128X4 ? kRows : kBlockRows, routing);
   if (s != NVFP4_OK) return s;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK) return s;
@@ -519,6 +530,32 @@ nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int
   if (s != NVFP4_OK) return s;
   return launch_quantize(routing, x_bf16, sum_M, K, num_groups, scratch, row_amax, row_amax, col_amax, out,
                          do_col, stream);
+}
+
+nvfp4_status nvfp4_row_post_scale(const float* gemm_out, int64_t rows, int64_t cols, const float* row_amax,
+                                  const float* bias, void* out, int32_t out_dtype, cudaStream_t stream) {
+  if (rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (gemm_out == nullptr || row_amax == nullptr || out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 4 != 0 || !aligned(gemm_out, 16) || !aligned(bias, 16) || !aligned(row_amax, 4) ||
+      !aligned(out, out_dtype == NVFP4_OUT_BF16 ? 8 : 16))
+    return NVFP4_ERR_UNSUPPORTED;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t units = (rows + kPostUnitRows - 1) / kPostUnitRows * ((cols / 4 + 31) / 32);
+  int64_t grid = (units + kPostThreads / 32 - 1) / (kPostThreads / 32);
+  const int64_t cap = static_cast<int64_t>(sms) * 2;  // persistent: two CTAs per SM are resident
+  if (grid > cap) grid = cap;
+  const bool b16 = out_dtype == NVFP4_OUT_BF16, has_bias = bias != nullptr;
+  auto kernel = b16 ? (has_bias ? row_post_scale_kernel<true, true> : row_post_scale_kernel<true, false>)
+                    : (has_bias ? row_post_scale_kernel<false, true> : row_post_scale_kernel<false, false>);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kPostThreads);
+  cfg.stream = stream;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, reinterpret_cast<const float4*>(gemm_out), rows, cols / 4,
+                                        row_amax, reinterpret_cast<const float4*>(bias), out));
 }
 
 const char* nvfp4_status_string(nvfp4_status status) {

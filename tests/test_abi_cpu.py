@@ -163,6 +163,23 @@ def test_quantize_noalloc_host_checks(L):
         abi.NVFP4_ERR_UNSUPPORTED  # beyond the static scratch
 
 
+def test_post_scale_host_checks(L):
+    f = L.nvfp4_row_post_scale
+    assert f(FAKE, 4, 6, FAKE, None, FAKE, abi.NVFP4_OUT_F32, None) == abi.NVFP4_ERR_UNSUPPORTED  # cols % 4
+    assert f(FAKE, 4, 8, FAKE, None, FAKE, 7, None) == abi.NVFP4_ERR_INVALID_ARG  # unknown dtype
+    assert f(None, 4, 8, FAKE, None, FAKE, abi.NVFP4_OUT_F32, None) == abi.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 4, 8, FAKE, None, ctypes.c_void_p(0x10008), abi.NVFP4_OUT_F32, None) == \
+        abi.NVFP4_ERR_UNSUPPORTED  # f32 output must be 16-byte aligned
+    assert f(FAKE, 0, 8, FAKE, None, FAKE, abi.NVFP4_OUT_BF16, None) == abi.NVFP4_OK  # empty
+
+
+def test_scale_layout_must_be_known(L):
+    arr = (ctypes.c_int64 * 1)(128)
+    o = abi.Outputs(row_data=0x10000, row_scale=0x10000, row_s2=0x10000, scale_layout=5)
+    assert L.nvfp4_group_cast(FAKE, 128, 128, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_INVALID_ARG
+
+
 def test_dequantize_host_checks(L):
     f = L.nvfp4_dequantize
     assert f(FAKE, FAKE, FAKE, 4, 24, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG
