@@ -76,6 +76,15 @@ def _declare(L):
     L.nvo_group_cast.restype = ctypes.c_int
     L.nvo_dequantize.argtypes = [_u8p, _u8p, _f32p, ctypes.c_int64, ctypes.c_int64, _f32p]
     L.nvo_dequantize.restype = ctypes.c_int
+    L.nvo_e8m0_decode.argtypes = [ctypes.c_uint8]
+    L.nvo_e8m0_decode.restype = ctypes.c_float
+    L.nvo_mx_block_encode.argtypes = [_f32p, _u8p, _u8p]
+    L.nvo_mx_block_encode.restype = None
+    L.nvo_mx_group_cast.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, _i64p, ctypes.c_int32,
+                                    _u8p, _u8p, _u8p, _u8p]
+    L.nvo_mx_group_cast.restype = ctypes.c_int
+    L.nvo_mx_dequantize.argtypes = [_u8p, _u8p, ctypes.c_int64, ctypes.c_int64, _f32p]
+    L.nvo_mx_dequantize.restype = ctypes.c_int
     L.nvo_swizzle_scales_128x4.argtypes = [_u8p, ctypes.c_int64, ctypes.c_int64, _u8p]
     L.nvo_swizzle_scales_128x4.restype = ctypes.c_int
     L.nvo_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -276,3 +285,49 @@ def swizzle_cast_scales(out: dict, m_splits: Sequence[int], K: int) -> dict:
                 parts.append(swizzle_scales_128x4(col_slice(cs, m_splits, K, g, 16), K, m // 16))
         res["col_scale"] = np.concatenate(parts) if parts else np.zeros(0, np.uint8)
     return res
+
+
+# -------------------------------------------------------------------- MXFP4
+
+def e8m0_decode(code: int) -> float:
+    return float(lib().nvo_e8m0_decode(int(code)))
+
+
+def mx_block_encode(x32: np.ndarray):
+    """(E8M0 scale byte, 32 codes) of one MXFP4 block."""
+    x32 = np.ascontiguousarray(x32, dtype=np.float32)
+    assert x32.size == 32
+    s8 = np.zeros(1, dtype=np.uint8)
+    codes = np.zeros(32, dtype=np.uint8)
+    lib().nvo_mx_block_encode(_ptr(x32, _f32p), _ptr(s8, _u8p), _ptr(codes, _u8p))
+    return int(s8[0]), codes
+
+
+def mx_group_cast(x: np.ndarray, m_splits: Sequence[int], rows: bool = True, cols: bool = True) -> dict:
+    """Grouped MXFP4 cast of bf16 bits x [sum_M, K]: row_data [sum_M, K/2],
+    row_scale [sum_M, K/32], col_data / col_scale flat (group g at K*o_g/2,
+    K*o_g/32, shapes [K, m_g/2], [K, m_g/32])."""
+    x = _x(x)
+    M, K = x.shape
+    sp = _splits(m_splits)
+    out = {}
+    if rows:
+        out["row_data"] = np.zeros((M, K // 2), dtype=np.uint8)
+        out["row_scale"] = np.zeros((M, K // 32), dtype=np.uint8)
+    if cols:
+        out["col_data"] = np.zeros(M * K // 2, dtype=np.uint8)
+        out["col_scale"] = np.zeros(M * K // 32, dtype=np.uint8)
+    rc = lib().nvo_mx_group_cast(_ptr(x, _u16p), M, K, _ptr(sp, _i64p), len(sp),
+                                 _ptr(out.get("row_data"), _u8p), _ptr(out.get("row_scale"), _u8p),
+                                 _ptr(out.get("col_data"), _u8p), _ptr(out.get("col_scale"), _u8p))
+    _check(rc, "mx_group_cast")
+    return out
+
+
+def mx_dequantize(data: np.ndarray, scale: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    data = np.ascontiguousarray(data, dtype=np.uint8).reshape(-1)
+    scale = np.ascontiguousarray(scale, dtype=np.uint8).reshape(-1)
+    out = np.zeros((rows, cols), dtype=np.float32)
+    _check(lib().nvo_mx_dequantize(_ptr(data, _u8p), _ptr(scale, _u8p), rows, cols, _ptr(out, _f32p)),
+           "mx_dequantize")
+    return out

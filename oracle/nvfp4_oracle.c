@@ -290,6 +290,96 @@ int nvo_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
   return NVO_OK;
 }
 
+/* ------------------------------------------------------------------- MXFP4 */
+
+/* [T] E8M0: an exponent byte with bias 127, no sign, no mantissa */
+float nvo_e8m0_decode(uint8_t code) {
+  if (code == 0xFF) return NAN;
+  return ldexpf(1.0f, (int)code - 127);
+}
+
+/* [T] one block of 32: the shared exponent from the block amax (frexp gives
+ * a = m * 2^k with m in [0.5, 1), so floor(log2 a) = k - 1 exactly), then
+ * every element scaled by the power of two and encoded */
+void nvo_mx_block_encode(const float* x32, uint8_t* e8m0, uint8_t* codes32) {
+  float a = 0.0f;
+  for (int i = 0; i < 32; i++) {
+    const float m = fabsf(x32[i]);
+    if (m > a) a = m;
+  }
+  int s = -127;
+  if (a > 0.0f) {
+    int k;
+    frexpf(a, &k);
+    s = (k - 1) - 2;
+    if (s < -127) s = -127;
+    if (s > 127) s = 127;
+  }
+  *e8m0 = (uint8_t)(s + 127);
+  for (int i = 0; i < 32; i++) codes32[i] = nvo_e2m1_encode(ldexpf(x32[i], -s));
+}
+
+int nvo_mx_group_cast(const uint16_t* x, int64_t sum_M, int64_t K, const int64_t* m_splits, int32_t E,
+                      uint8_t* row_data, uint8_t* row_scale, uint8_t* col_data, uint8_t* col_scale) {
+  if (sum_M < 0 || K < 0 || E < 0 || (K % 32) != 0) return NVO_E_ARG;
+  if (E > 0 && m_splits == NULL) return NVO_E_ARG;
+  const int do_row = row_data != NULL || row_scale != NULL;
+  const int do_col = col_data != NULL || col_scale != NULL;
+  int64_t total = 0;
+  for (int32_t g = 0; g < E; g++) {
+    if (m_splits[g] < 0 || (do_col && (m_splits[g] % 32) != 0)) return NVO_E_ARG;
+    total += m_splits[g];
+  }
+  if (total != sum_M) return NVO_E_ARG;
+  if (sum_M * K > 0 && x == NULL) return NVO_E_ARG;
+  if (do_row && sum_M * K > 0 && (row_data == NULL || row_scale == NULL)) return NVO_E_ARG;
+  if (do_col && sum_M * K > 0 && (col_data == NULL || col_scale == NULL)) return NVO_E_ARG;
+  for (int64_t i = 0; i < sum_M * K; i++)
+    if (!isfinite(nvo_bf16_to_f32(x[i]))) return NVO_E_NONFINITE;
+  float blk[32];
+  uint8_t codes[32];
+  if (do_row) {
+    for (int64_t r = 0; r < sum_M; r++) {
+      for (int64_t b = 0; b < K / 32; b++) {
+        for (int i = 0; i < 32; i++) blk[i] = nvo_bf16_to_f32(x[r * K + b * 32 + i]);
+        nvo_mx_block_encode(blk, &row_scale[r * (K / 32) + b], codes);
+        for (int i = 0; i < 32; i += 2)
+          row_data[r * (K / 2) + b * 16 + i / 2] = (uint8_t)(codes[i] | (codes[i + 1] << 4));
+      }
+    }
+  }
+  if (do_col) {
+    int64_t o = 0;
+    for (int32_t g = 0; g < E; g++) {
+      const int64_t m = m_splits[g];
+      uint8_t* cd = col_data + K * o / 2;
+      uint8_t* cs = col_scale + K * o / 32;
+      for (int64_t k = 0; k < K; k++) {
+        for (int64_t b = 0; b < m / 32; b++) {
+          for (int i = 0; i < 32; i++) blk[i] = nvo_bf16_to_f32(x[(o + b * 32 + i) * K + k]);
+          nvo_mx_block_encode(blk, &cs[k * (m / 32) + b], codes);
+          for (int i = 0; i < 32; i += 2) cd[k * (m / 2) + b * 16 + i / 2] = (uint8_t)(codes[i] | (codes[i + 1] << 4));
+        }
+      }
+      o += m;
+    }
+  }
+  return NVO_OK;
+}
+
+int nvo_mx_dequantize(const uint8_t* data, const uint8_t* scale, int64_t rows, int64_t cols, float* out) {
+  if (rows < 0 || cols < 0 || (cols % 32) != 0) return NVO_E_ARG;
+  if (rows * cols > 0 && (data == NULL || scale == NULL || out == NULL)) return NVO_E_ARG;
+  for (int64_t r = 0; r < rows; r++) {
+    for (int64_t c = 0; c < cols; c++) {
+      const uint8_t byte = data[r * (cols / 2) + c / 2];
+      const uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      out[r * cols + c] = nvo_e2m1_decode(code) * nvo_e8m0_decode(scale[r * (cols / 32) + c / 32]);
+    }
+  }
+  return NVO_OK;
+}
+
 /* ------------------------------------------------ consumer side of the cast */
 
 /* [T] the 128x4-tiled scale layout, written straight from its index map */

@@ -91,6 +91,31 @@ int nvo_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
  * ceil(rows/128)*128 * ceil(cols/4)*4 bytes. */
 int nvo_swizzle_scales_128x4(const uint8_t* scale, int64_t rows, int64_t cols, uint8_t* out);
 
+/* ------------------------------------------------------------- MXFP4 */
+
+/* MXFP4: E2M1 data in blocks of 32 elements with one E8M0 (power-of-two)
+ * scale each and no second-level scale (TransformerEngine #3824, Testing and
+ * item 1: the "E2M1/block-32/E8M0" pow_2_scales configuration; row-scaled
+ * NVFP4 is not combined with it). The pages do not spell out the scale
+ * rule; reading (the OCP Microscaling conversion): with a = max |x| of the
+ * block, the shared exponent is s = floor(log2 a) - 2 (2 = exponent of
+ * E2M1's largest value, 6 = 1.5 * 2^2), clamped to [-127, 127] (a = 0 gives
+ * -127); the scale byte is s + 127; each element encodes as
+ * E2M1_rne_satfinite(x * 2^-s) (exact multiply; values past 6 saturate). */
+float nvo_e8m0_decode(uint8_t code);  /* 2^(code-127); NaN for 0xFF */
+void nvo_mx_block_encode(const float* x32, uint8_t* e8m0, uint8_t* codes32);
+
+/* grouped MXFP4 cast: rowwise row_data [sum_M, K/2], row_scale [sum_M, K/32];
+ * colwise per group g col_data at byte K*o_g/2 of shape [K, m_g/2] and
+ * col_scale at byte K*o_g/32 of shape [K, m_g/32]. K % 32 == 0, and for the
+ * colwise direction every m_g % 32 == 0. A direction whose two pointers are
+ * NULL is skipped. */
+int nvo_mx_group_cast(const uint16_t* x, int64_t sum_M, int64_t K, const int64_t* m_splits, int32_t E,
+                      uint8_t* row_data, uint8_t* row_scale, uint8_t* col_data, uint8_t* col_scale);
+
+/* x_hat = e2m1(code) * 2^(scale-127), one row-major matrix [rows, cols] */
+int nvo_mx_dequantize(const uint8_t* data, const uint8_t* scale, int64_t rows, int64_t cols, float* out);
+
 /* IEEE binary32 -> bfloat16 bits, round to nearest even (NaN stays NaN). */
 uint16_t nvo_f32_to_bf16(float v);
 
