@@ -344,6 +344,19 @@ def main():
     post_bytes = M * POST_N * (4 + 2) + 4 * M + 4 * POST_N
     del gemm_out, post_out
 
+    # ---- MXFP4 cast of the same input (one launch, both directions)
+    mx_out = abi.alloc_mx_outputs(M, K, dev)
+
+    def mx_step():
+        abi.nvfp4_mx_group_cast(x, splits, mx_out)
+
+    for _ in range(args.warmup):
+        mx_step()
+    barrier()
+    mx_ms = max_over_ranks(timed(mx_step, args.steps), world, dev)
+    mx_bytes = 2 * N + 2 * (N // 2 + N // 32)
+    del mx_out
+
     # ---- end to end through the C ABI with host buffers (pinned)
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
     e2e_steps = max(3, min(args.steps, 5))
@@ -443,6 +456,13 @@ def main():
                 "hbm_gbs": round(post_bytes / (post_ms * 1e-3) / 1e9, 1),
                 "hbm_frac_of_peak": round(post_bytes / (post_ms * 1e-3) / 1e9 / peak, 4),
             },
+        },
+        "mxfp4": {
+            "path": "nvfp4_mx_group_cast (E2M1, 32-element blocks, E8M0 scales), rowwise + colwise",
+            "ms_per_step": round(mx_ms, 4),
+            "value": round(job_throughput(N, world, mx_ms), 3),
+            "hbm_gbs": round(mx_bytes / (mx_ms * 1e-3) / 1e9, 1),
+            "hbm_frac_of_peak": round(mx_bytes / (mx_ms * 1e-3) / 1e9 / peak, 4),
         },
         "gpu_launches": 2 * args.steps,
         "clocks": clk,

@@ -299,6 +299,46 @@ NVFP4RS_API nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_
 NVFP4RS_API nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
                               int64_t rows, int64_t cols, float* out_f32, cudaStream_t stream);
 
+/* ------------------------------------------------------------------ MXFP4
+ * MXFP4: E2M1 data, blocks of 32 elements, one E8M0 (power-of-two) scale per
+ * block, no second-level scale (TransformerEngine #3824, Testing and item 1:
+ * the "E2M1/block-32/E8M0" pow_2_scales configuration, which row-scaled
+ * NVFP4 is not combined with). Scale rule (OCP Microscaling conversion; the
+ * pages do not spell it out): with a = max |x| of the block,
+ *   s = clamp(floor(log2 a) - 2, -127, 127)   (a == 0 gives -127)
+ *   scale byte = s + 127;  code_j = E2M1_rne_satfinite(x_j * 2^-s), sign kept
+ *   dequantize: x_hat = e2m1(code) * 2^(scale - 127)
+ * Same grouped structure as the NVFP4 cast; groups must be multiples of 128
+ * rows and K % 128 == 0 (else NVFP4_ERR_UNSUPPORTED). One read of x, one
+ * launch: no amax step. */
+typedef struct {
+  uint8_t* row_data;  /* [rows, K/2]                               */
+  uint8_t* row_scale; /* [rows, K/32] E8M0                         */
+  uint8_t* col_data;  /* per group [K, m_g/2] at byte K*o_g/2      */
+  uint8_t* col_scale; /* per group [K, m_g/32] at byte K*o_g/32    */
+} nvfp4_mx_outputs;
+
+/* Grouped MXFP4 cast, host-split routing (arguments as nvfp4_group_cast). */
+NVFP4RS_API nvfp4_status nvfp4_mx_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
+                                 const int64_t* m_splits_host, int32_t num_groups,
+                                 const nvfp4_mx_outputs* out, cudaStream_t stream);
+
+/* Grouped MXFP4 cast, graph-safe routing (arguments and status as
+ * nvfp4_group_cast_graphsafe; a group that is not a multiple of 128 rows is
+ * NVFP4_ERR_UNSUPPORTED on the device). Byte-identical to the host-split call. */
+NVFP4RS_API nvfp4_status nvfp4_mx_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                           const int64_t* first_dims_dev,
+                                           const int64_t* tensor_offsets_dev, int32_t num_groups,
+                                           const nvfp4_mx_outputs* out, int32_t* status_dev,
+                                           cudaStream_t stream);
+
+/* Decode one MXFP4 matrix [rows, cols]: data [rows, cols/2], scale
+ * [rows, cols/32] -> out fp32 [rows, cols]. cols % 32 == 0 (else
+ * NVFP4_ERR_INVALID_ARG); data and out 16-byte aligned (else
+ * NVFP4_ERR_UNSUPPORTED). Colwise output of group g: rows = K, cols = m_g. */
+NVFP4RS_API nvfp4_status nvfp4_mx_dequantize(const uint8_t* data, const uint8_t* scale, int64_t rows,
+                                 int64_t cols, float* out_f32, cudaStream_t stream);
+
 /* Output type of nvfp4_row_post_scale. */
 typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
 

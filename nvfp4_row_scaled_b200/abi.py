@@ -54,6 +54,12 @@ class Outputs(ctypes.Structure):
                 ("scale_layout", ctypes.c_int32)]
 
 
+class MxOutputs(ctypes.Structure):
+    """Mirror of ``nvfp4_mx_outputs``."""
+    _fields_ = [("row_data", ctypes.c_void_p), ("row_scale", ctypes.c_void_p),
+                ("col_data", ctypes.c_void_p), ("col_scale", ctypes.c_void_p)]
+
+
 def lib():
     """Open the library (once). Raises if it has not been built."""
     global _lib
@@ -76,6 +82,12 @@ def lib():
                                            vp, sz, vp]
         L.nvfp4_group_quantize_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp,
                                                      ctypes.POINTER(Outputs), vp, sz, vp, vp]
+        L.nvfp4_mx_group_cast.argtypes = [vp, i64, i64, vp, i32, ctypes.POINTER(MxOutputs), vp]
+        L.nvfp4_mx_group_cast_graphsafe.argtypes = [vp, i64, i64, vp, vp, i32, ctypes.POINTER(MxOutputs),
+                                                    vp, vp]
+        L.nvfp4_mx_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
+        for f in ("nvfp4_mx_group_cast", "nvfp4_mx_group_cast_graphsafe", "nvfp4_mx_dequantize"):
+            getattr(L, f).restype = ctypes.c_int
         L.nvfp4_row_post_scale.argtypes = [vp, i64, i64, vp, vp, vp, i32, vp]
         L.nvfp4_row_post_scale.restype = ctypes.c_int
         L.nvfp4_group_quantize_noalloc.argtypes = [vp, i64, i64, vp, i32, vp, vp,
@@ -262,6 +274,55 @@ def nvfp4_row_post_scale(gemm_out: torch.Tensor, row_amax: torch.Tensor, out: to
                                     _dev(bias, torch.float32, "bias"), _dev(out, out.dtype, "out"), dt,
                                     _stream(stream))
     _check(rc, "nvfp4_row_post_scale")
+
+
+def _mx_outputs(out: Dict[str, torch.Tensor]) -> MxOutputs:
+    o = MxOutputs()
+    for name in ("row_data", "row_scale", "col_data", "col_scale"):
+        p = _dev(out.get(name), torch.uint8, name)
+        setattr(o, name, p.value if p is not None else None)
+    return o
+
+
+def nvfp4_mx_group_cast(x: torch.Tensor, m_splits: Sequence[int], out: Dict[str, torch.Tensor],
+                        stream=None) -> None:
+    arr, E = _splits(m_splits)
+    o = _mx_outputs(out)
+    rc = lib().nvfp4_mx_group_cast(_dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1], arr, E,
+                                   ctypes.byref(o), _stream(stream))
+    _check(rc, "nvfp4_mx_group_cast")
+
+
+def nvfp4_mx_group_cast_graphsafe(x: torch.Tensor, first_dims: Optional[torch.Tensor],
+                                  tensor_offsets: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
+                                  status: torch.Tensor, stream=None,
+                                  num_groups: Optional[int] = None) -> None:
+    o = _mx_outputs(out)
+    rc = lib().nvfp4_mx_group_cast_graphsafe(
+        _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
+        _dev(first_dims, torch.int64, "first_dims"), _dev(tensor_offsets, torch.int64, "tensor_offsets"),
+        _groups(first_dims, num_groups), ctypes.byref(o), _dev(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "nvfp4_mx_group_cast_graphsafe")
+
+
+def nvfp4_mx_dequantize(data: torch.Tensor, scale: torch.Tensor, rows: int, cols: int, out: torch.Tensor,
+                        stream=None) -> None:
+    rc = lib().nvfp4_mx_dequantize(_dev(data, torch.uint8, "data"), _dev(scale, torch.uint8, "scale"),
+                                   int(rows), int(cols), _dev(out, torch.float32, "out"), _stream(stream))
+    _check(rc, "nvfp4_mx_dequantize")
+
+
+def alloc_mx_outputs(rows: int, K: int, device="cuda", row: bool = True,
+                     col: bool = True) -> Dict[str, torch.Tensor]:
+    """Uninitialised output buffers of the grouped MXFP4 cast for ``rows`` rows."""
+    out: Dict[str, torch.Tensor] = {}
+    if row:
+        out["row_data"] = torch.empty(rows, K // 2, dtype=torch.uint8, device=device)
+        out["row_scale"] = torch.empty(rows, K // 32, dtype=torch.uint8, device=device)
+    if col:
+        out["col_data"] = torch.empty(rows * K // 2, dtype=torch.uint8, device=device)
+        out["col_scale"] = torch.empty(rows * K // 32, dtype=torch.uint8, device=device)
+    return out
 
 
 def nvfp4_dequantize(data: torch.Tensor, scale: torch.Tensor, s2: torch.Tensor, rows: int, cols: int,

@@ -190,6 +190,69 @@ __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
 // stores and the staging of the other outputs. kExact selects the
 // IEEE-divide block scales (tiles with a row or column amax outside the
 // shortcut's range).
+// The codes of a lane's 16 x 8 patch, once the multipliers are known: renc[i]
+// multiplies row i (rowwise codes, stored straight to rdst + i * row_pitch
+// when row_store), cenc2[q] the column pair (2q, 2q+1) (colwise codes, staged
+// transposed in st.col_data: 8 bytes per column at slot rb ^ (cc % 8)). Shared
+// by the NVFP4 and the MXFP4 casts.
+__device__ __forceinline__ void encode_codes(const uint4 (&v)[16], const float (&renc)[16],
+                                             const uint64_t (&cenc2)[4], CastStage& st, bool do_row,
+                                             bool do_col, int cc, int rb, uint8_t* rdst, size_t row_pitch,
+                                             bool row_store) {
+  const int slot = rb ^ (cc & 7);
+#pragma unroll
+  for (int half = 0; half < 2; half++) {
+    uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
+#pragma unroll
+    for (int pp = 0; pp < 4; pp++) {
+      const int i = 8 * half + 2 * pp;
+      const uint64_t x0[4] = {unpack2(v[i].x), unpack2(v[i].y), unpack2(v[i].z), unpack2(v[i].w)};
+      const uint64_t x1[4] = {unpack2(v[i + 1].x), unpack2(v[i + 1].y), unpack2(v[i + 1].z),
+                              unpack2(v[i + 1].w)};
+      if (do_row) {
+        const uint64_t e0 = pack2(renc[i], renc[i]), e1 = pack2(renc[i + 1], renc[i + 1]);
+        const uint32_t w0 = e2m1_pairs(mul2x(x0[0], e0), mul2x(x0[1], e0), mul2x(x0[2], e0), mul2x(x0[3], e0));
+        const uint32_t w1 = e2m1_pairs(mul2x(x1[0], e1), mul2x(x1[1], e1), mul2x(x1[2], e1), mul2x(x1[3], e1));
+        if (row_store) {  // false for a 16-row block past the routed rows
+          st_global_u32(rdst + i * row_pitch, w0);
+          st_global_u32(rdst + (i + 1) * row_pitch, w1);
+        }
+      }
+      if (do_col) {
+        uint64_t y0[4], y1[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          y0[q] = mul2x(x0[q], cenc2[q]);
+          y1[q] = mul2x(x1[q], cenc2[q]);
+        }
+        // byte q of A = codes of (row i, row i+1) in column q
+        A[pp] = e2m1_cross(y0[0], y1[0], y0[1], y1[1]);
+        B[pp] = e2m1_cross(y0[2], y1[2], y0[3], y1[3]);
+      }
+    }
+    if (do_col) {
+      // 4x4 byte transposes: the word of column q = bytes A[0..3][q], rows
+      // 8*half .. 8*half+7 of this lane's block, staged right away
+      uint32_t cw[8];
+      const uint32_t t0 = prmt(A[0], A[1], 0x5140), t1 = prmt(A[0], A[1], 0x7362);
+      const uint32_t t2 = prmt(A[2], A[3], 0x5140), t3 = prmt(A[2], A[3], 0x7362);
+      cw[0] = prmt(t0, t2, 0x5410);
+      cw[1] = prmt(t0, t2, 0x7632);
+      cw[2] = prmt(t1, t3, 0x5410);
+      cw[3] = prmt(t1, t3, 0x7632);
+      const uint32_t u0 = prmt(B[0], B[1], 0x5140), u1 = prmt(B[0], B[1], 0x7362);
+      const uint32_t u2 = prmt(B[2], B[3], 0x5140), u3 = prmt(B[2], B[3], 0x7362);
+      cw[4] = prmt(u0, u2, 0x5410);
+      cw[5] = prmt(u0, u2, 0x7632);
+      cw[6] = prmt(u1, u3, 0x5410);
+      cw[7] = prmt(u1, u3, 0x7632);
+#pragma unroll
+      for (int q = 0; q < 8; q++)
+        *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
+    }
+  }
+}
+
 // The shared tables a tile's encode reads: {value, RN(1/value)} of every
 // E4M3 code, and S_enc of the tile's 128 rows and 128 columns.
 struct EncodeTables {
@@ -269,58 +332,7 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
   }
 
   // -------------------------------------------------------------- codes
-  const int slot = rb ^ (cc & 7);
-#pragma unroll
-  for (int half = 0; half < 2; half++) {
-    uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
-#pragma unroll
-    for (int pp = 0; pp < 4; pp++) {
-      const int i = 8 * half + 2 * pp;
-      const uint64_t x0[4] = {unpack2(v[i].x), unpack2(v[i].y), unpack2(v[i].z), unpack2(v[i].w)};
-      const uint64_t x1[4] = {unpack2(v[i + 1].x), unpack2(v[i + 1].y), unpack2(v[i + 1].z),
-                              unpack2(v[i + 1].w)};
-      if (do_row) {
-        const uint64_t e0 = pack2(renc[i], renc[i]), e1 = pack2(renc[i + 1], renc[i + 1]);
-        const uint32_t w0 = e2m1_pairs(mul2x(x0[0], e0), mul2x(x0[1], e0), mul2x(x0[2], e0), mul2x(x0[3], e0));
-        const uint32_t w1 = e2m1_pairs(mul2x(x1[0], e1), mul2x(x1[1], e1), mul2x(x1[2], e1), mul2x(x1[3], e1));
-        if (row_store) {  // false for a 16-row block past the routed rows
-          st_global_u32(rdst + i * row_pitch, w0);
-          st_global_u32(rdst + (i + 1) * row_pitch, w1);
-        }
-      }
-      if (do_col) {
-        uint64_t y0[4], y1[4];
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          y0[q] = mul2x(x0[q], cenc2[q]);
-          y1[q] = mul2x(x1[q], cenc2[q]);
-        }
-        // byte q of A = codes of (row i, row i+1) in column q
-        A[pp] = e2m1_cross(y0[0], y1[0], y0[1], y1[1]);
-        B[pp] = e2m1_cross(y0[2], y1[2], y0[3], y1[3]);
-      }
-    }
-    if (do_col) {
-      // 4x4 byte transposes: the word of column q = bytes A[0..3][q], rows
-      // 8*half .. 8*half+7 of this lane's block, staged right away
-      uint32_t cw[8];
-      const uint32_t t0 = prmt(A[0], A[1], 0x5140), t1 = prmt(A[0], A[1], 0x7362);
-      const uint32_t t2 = prmt(A[2], A[3], 0x5140), t3 = prmt(A[2], A[3], 0x7362);
-      cw[0] = prmt(t0, t2, 0x5410);
-      cw[1] = prmt(t0, t2, 0x7632);
-      cw[2] = prmt(t1, t3, 0x5410);
-      cw[3] = prmt(t1, t3, 0x7632);
-      const uint32_t u0 = prmt(B[0], B[1], 0x5140), u1 = prmt(B[0], B[1], 0x7362);
-      const uint32_t u2 = prmt(B[2], B[3], 0x5140), u3 = prmt(B[2], B[3], 0x7362);
-      cw[4] = prmt(u0, u2, 0x5410);
-      cw[5] = prmt(u0, u2, 0x7632);
-      cw[6] = prmt(u1, u3, 0x5410);
-      cw[7] = prmt(u1, u3, 0x7632);
-#pragma unroll
-      for (int q = 0; q < 8; q++)
-        *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
-    }
-  }
+  encode_codes(v, renc, cenc2, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
 }
 
 // The 128x4-tiled scale layout (the grouped GEMM's swizzle contract; see the
@@ -346,23 +358,30 @@ __device__ __forceinline__ uint2 tiled_piece(const uint8_t* stg, int t) {
 // Stores of the outputs a tile staged: colwise data (64 bytes per column,
 // four 16-byte pieces), colwise scales (8 bytes per column) and rowwise scales
 // (8 bytes per row), all with the L2 evict-last policy `keep`.
+// The staged colwise codes of a whole tile of a 128-aligned group: 64 bytes
+// per column (four 16-byte pieces) into the group's transposed slice.
+__device__ __forceinline__ void store_col_data(const CastStage& st, uint8_t* col_data, int K, int32_t o_g,
+                                               int64_t m_g, int32_t r0, int c0, int t, uint64_t keep) {
+  const size_t half_m = static_cast<size_t>(m_g) >> 1;
+  uint8_t* gd = col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
+#pragma unroll
+  for (int kk = 0; kk < 4; kk++) {
+    const int u = kk * kCastThreads + t;
+    const int col = u >> 2, part = u & 3;
+    const int sw = (col >> 3) & 7;
+    const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
+    const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
+    st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part, make_uint4(lo.x, lo.y, hi.x, hi.y),
+                      keep);
+  }
+}
+
 template <bool kTiled>
 __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut& out, int K,
                                              int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
                                              bool do_row, bool do_col, uint64_t keep) {
   if (do_col) {
-    const size_t half_m = static_cast<size_t>(m_g) >> 1;
-    uint8_t* gd = out.col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
-#pragma unroll
-    for (int kk = 0; kk < 4; kk++) {
-      const int u = kk * kCastThreads + t;
-      const int col = u >> 2, part = u & 3;
-      const int sw = (col >> 3) & 7;
-      const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
-      const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
-      st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part,
-                        make_uint4(lo.x, lo.y, hi.x, hi.y), keep);
-    }
+    store_col_data(st, out.col_data, K, o_g, m_g, r0, c0, t, keep);
     if (kTiled) {
       // the tile's 128 x 8 block scales are two whole 128x4 tiles of the
       // group's [K, m_g/16] scale matrix: tile row c0/128, tile columns

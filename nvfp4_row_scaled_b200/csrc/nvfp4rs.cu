@@ -24,6 +24,7 @@
 #include "group_quantize.cuh"
 #include "dequant.cuh"
 #include "post_scale.cuh"
+#include "mx_cast.cuh"
 
 using namespace nvfp4rs;
 
@@ -327,6 +328,51 @@ uint32_t* noalloc_scratch() {
   return addr[dev];
 }
 
+// MXFP4 output descriptor checks (like check_outputs: a direction is
+// requested when either of its pointers is set, then both must be set).
+nvfp4_status check_mx_outputs(const nvfp4_mx_outputs* out, int64_t rows, int64_t K, bool& do_row, bool& do_col) {
+  if (out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  do_row = out->row_data != nullptr || out->row_scale != nullptr;
+  do_col = out->col_data != nullptr || out->col_scale != nullptr;
+  const bool has_rows = rows > 0 && K > 0;
+  if (has_rows && ((do_row && (out->row_data == nullptr || out->row_scale == nullptr)) ||
+                   (do_col && (out->col_data == nullptr || out->col_scale == nullptr))))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(out->row_data, 16) || !aligned(out->row_scale, 16) || !aligned(out->col_data, 16) ||
+      !aligned(out->col_scale, 16))
+    return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+template <class Routing>
+nvfp4_status launch_mx_cast(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
+                            const nvfp4_mx_outputs* out, cudaStream_t stream) {
+  const int64_t tiles = (rows / kRows) * (K / kCols);
+  if (tiles == 0) return NVFP4_OK;
+  CUtensorMap map;
+  if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
+  auto kernel = mx_cast_kernel<Routing>;
+  const size_t smem = cast_smem_bytes(E) + 1024;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCastThreads, smem) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
+  int64_t grid = static_cast<int64_t>(sms) * per_sm;
+  if (tiles < grid) grid = tiles;
+  const MxOut o{out->row_data, out->row_scale, out->col_data, out->col_scale};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kCastThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), o));
+}
+
 }  // namespace
 
 extern "C" {
@@ -556,6 +602,57 @@ nvfp4_status nvfp4_row_post_scale(const float* gemm_out, int64_t rows, int64_t c
   cfg.stream = stream;
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, reinterpret_cast<const float4*>(gemm_out), rows, cols / 4,
                                         row_amax, reinterpret_cast<const float4*>(bias), out));
+}
+
+nvfp4_status nvfp4_mx_group_cast(const void* x_bf16, int64_t sum_M, int64_t K, const int64_t* m_splits_host,
+                                 int32_t num_groups, const nvfp4_mx_outputs* out, cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_mx_outputs(out, sum_M, K, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  static thread_local HostRouting routing;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kRows);
+  if (s != NVFP4_OK) return s;
+  if (!do_row && !do_col) return NVFP4_OK;
+  return launch_mx_cast(routing, x_bf16, sum_M, K, num_groups, out, stream);
+}
+
+nvfp4_status nvfp4_mx_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
+                                           const int64_t* first_dims_dev, const int64_t* tensor_offsets_dev,
+                                           int32_t num_groups, const nvfp4_mx_outputs* out, int32_t* status_dev,
+                                           cudaStream_t stream) {
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
+  if (s != NVFP4_OK) return s;
+  bool do_row = false, do_col = false;
+  s = check_mx_outputs(out, capacity_rows, K, do_row, do_col);
+  if (s != NVFP4_OK) return s;
+  DeviceRouting routing;
+  s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups, kRows,
+                     routing);
+  if (s != NVFP4_OK) return s;
+  s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
+  if (s != NVFP4_OK || K == 0 || (!do_row && !do_col)) return s;
+  return launch_mx_cast(routing, x_bf16, capacity_rows, K, num_groups, out, stream);
+}
+
+nvfp4_status nvfp4_mx_dequantize(const uint8_t* data, const uint8_t* scale, int64_t rows, int64_t cols,
+                                 float* out_f32, cudaStream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (data == nullptr || scale == nullptr || out_f32 == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(data, 16) || !aligned(out_f32, 16)) return NVFP4_ERR_UNSUPPORTED;
+  const int64_t blocks = rows * (cols / 32);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t grid = (blocks + kMxDequantThreads - 1) / kMxDequantThreads;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kMxDequantThreads);
+  cfg.stream = stream;
+  return cuda_status(cudaLaunchKernelEx(&cfg, mx_dequant_kernel, reinterpret_cast<const uint4*>(data), scale, blocks,
+                                        reinterpret_cast<float4*>(out_f32)));
 }
 
 const char* nvfp4_status_string(nvfp4_status status) {

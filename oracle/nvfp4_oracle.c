@@ -373,7 +373,7 @@ int nvo_mx_dequantize(const uint8_t* data, const uint8_t* scale, int64_t rows, i
   for (int64_t r = 0; r < rows; r++) {
     for (int64_t c = 0; c < cols; c++) {
       const uint8_t byte = data[r * (cols / 2) + c / 2];
-      const uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      const uint8_t code = (uint8_t)((byte >> (4 * (c % 2))) & 0xF); /* element 2j: low nibble */
       out[r * cols + c] = nvo_e2m1_decode(code) * nvo_e8m0_decode(scale[r * (cols / 32) + c / 32]);
     }
   }
