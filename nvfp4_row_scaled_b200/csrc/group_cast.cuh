@@ -77,6 +77,9 @@ struct CastSmem {
   float2 e4m3[128];                   // {value, RN(1/value)} per E4M3 code
   float row_senc[kRows];
   float col_senc[kRows / kBlockRows][kCols];  // per 16-row block: [0] only, unless the tile is mixed
+  float pf_col[kStages][kCols];  // plain kernel: the stage's tile's column amax (bulk copy)
+  float pf_row[kStages][kRows];  // its row amax, when it starts a new row tile for this CTA
+  int pf_g[kStages];             // its group
   uint64_t full[kStages];
 };
 
@@ -162,6 +165,36 @@ __device__ __forceinline__ void issue_tile_at(CastSmem& sm, const CUtensorMap* m
   mbar_expect_tx(&sm.full[s], kTileBytes);
   tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s], policy);
   tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s], policy);
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned, multiple of 16 bytes),
+// completion counted on `bar`. No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Plain cast kernel: tile `tl` into stage s together with what its encode
+// scales need -- its group, the 128 column amax of that group and, when the
+// tile starts a new row tile for this CTA, the 128 row amax -- by bulk copies
+// completing on the tile's own mbarrier, so the values arrive with the tile
+// (thread 0 only; amax pointers NULL for a direction not requested).
+__device__ __forceinline__ void issue_tile_amax(CastSmem& sm, const CUtensorMap* map, int s, int tl, int n_ct,
+                                                const RoutingSmem& rs, int K, const float* row_amax,
+                                                const float* col_amax, bool new_row) {
+  const int rt = tl / n_ct, ct = tl - rt * n_ct;
+  const int g = group_of_row(rs, rt * kRows);
+  sm.pf_g[s] = g;
+  const bool rows = row_amax != nullptr && new_row;
+  mbar_expect_tx(&sm.full[s], kTileBytes + (col_amax != nullptr ? 512u : 0u) + (rows ? 512u : 0u));
+  const uint64_t pol = policy_evict_first();
+  tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s], pol);
+  tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s], pol);
+  if (col_amax != nullptr) bulk_load(sm.pf_col[s], col_amax + static_cast<size_t>(g) * K + ct * kCols, 512u, &sm.full[s]);
+  if (rows) bulk_load(sm.pf_row[s], row_amax + static_cast<size_t>(rt) * kRows, 512u, &sm.full[s]);
 }
 
 // Tile number `tl` of the row-major tile order (read once: evict first).
@@ -513,8 +546,13 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   }
   __syncthreads();
   if (t == 0) {
-    for (int s = 0; s < kStages && blockIdx.x + s * G < n_tiles; s++)
-      issue_tile(sm, &tmap, s, blockIdx.x + s * G, n_ct);
+    for (int s = 0; s < kStages && blockIdx.x + s * G < n_tiles; s++) {
+      const int tl = blockIdx.x + s * G;
+      if (kGeneral)
+        issue_tile(sm, &tmap, s, tl, n_ct);
+      else
+        issue_tile_amax(sm, &tmap, s, tl, n_ct, rs, K, do_row ? row_amax : nullptr, do_col ? col_amax : nullptr, s == 0 || (tl - G) / n_ct != tl / n_ct);
+    }
   }
 
   const int lane = t & 31, warp = t >> 5;
@@ -540,24 +578,27 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     if (t == 0) slow_tile[(k + 1) & 1] = 0;  // flag of the next tile (last read a tile ago)
     bool slow = false;
     const int valid = kGeneral ? min(kRows, rs.total - r0) : kRows;  // routed rows (a multiple of 16)
+    // plain kernel: the tile's amax values come with it (issue_tile_amax)
+    bool ok = true;
+    if (!kGeneral) ok = mbar_wait(&sm.full[s], phase);
     if (rt != cur_rt) {  // new row tile: its group(s) and its rows' encode scales
       cur_rt = rt;
-      g = group_of_row(rs, r0);
+      g = kGeneral ? group_of_row(rs, r0) : sm.pf_g[s];
       o_g = rs.off[g];
       m_g = rs.off[g + 1] - o_g;
       if (do_row) {
         const bool in = t < valid;
-        const float a = in ? row_amax[r0 + t] : 0.0f;
+        const float a = in ? (kGeneral ? row_amax[r0 + t] : sm.pf_row[s][t]) : 0.0f;
         sm.row_senc[t] = s_enc_of(a);
         row_slow = in && !fast_path_amax(a);
-        if (ct == 0 && in) out.row_s2[r0 + t] = s_dec_of(a);
+        if (ct == 0 && in && ok) out.row_s2[r0 + t] = s_dec_of(a);
       }
     }
     slow |= row_slow;
     const bool mixed = kGeneral && o_g + m_g < r0 + valid;  // the tile crosses a group boundary
     if (do_col) {
       if (!mixed) {
-        const float a = col_amax[static_cast<size_t>(g) * K + c0 + t];
+        const float a = kGeneral ? col_amax[static_cast<size_t>(g) * K + c0 + t] : sm.pf_col[s][t];
         sm.col_senc[0][t] = s_enc_of(a);
         slow |= !fast_path_amax(a);
       } else {  // one column table per 16-row block, from the block's group
@@ -572,7 +613,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     if (slow) slow_tile[k & 1] = 1;
 
     // this lane's 16 x 8 patch from the swizzled stage
-    const bool ok = mbar_wait(&sm.full[s], phase);
+    if (kGeneral) ok = mbar_wait(&sm.full[s], phase);
     uint4 v[16];
     load_patch(sm.tile[s], cc, rl, v);
     if (__syncthreads_or(!ok)) {
@@ -583,7 +624,11 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     // this barrier: refill it with tile k+1 (tiles 0 and 1 came in the prologue).
     if (t == 0 && k >= 1 && tl + G < n_tiles) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
+      if (kGeneral)
+        issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
+      else
+        issue_tile_amax(sm, &tmap, (k + 1) % kStages, tl + G, n_ct, rs, K, do_row ? row_amax : nullptr, do_col ? col_amax : nullptr,
+                        (tl + G) / n_ct != rt);
     }
     // stage s is free once every thread holds its patch: it stages the outputs
     CastStage& st = *reinterpret_cast<CastStage*>(sm.tile[s]);

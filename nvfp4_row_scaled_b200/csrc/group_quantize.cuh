@@ -178,16 +178,6 @@ __device__ __forceinline__ bool mbar_wait_flag(uint64_t* bar, uint32_t phase, co
   return false;
 }
 
-// Untiled bulk copy global -> shared (16-byte aligned, multiple of 16 bytes),
-// completion counted on `bar`. No multicast.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
 // Compute warps' named barrier (warps 0-3); returns the OR of `pred` over them.
 __device__ __forceinline__ bool compute_bar_or(bool pred) {
   uint32_t r;

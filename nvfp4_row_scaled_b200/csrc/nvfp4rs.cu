@@ -408,6 +408,8 @@ nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
   if ((do_row && sum_M > 0 && row_amax == nullptr) ||
       (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
     return NVFP4_ERR_INVALID_ARG;
+  // the cast copies 512-byte runs of both amax vectors with the TMA unit
+  if (!aligned(row_amax, 16) || !aligned(col_amax, 16)) return NVFP4_ERR_UNSUPPORTED;
   static thread_local HostRouting routing;
   bool all_128 = true;
   s = host_routing(m_splits_host, num_groups, sum_M, routing, kBlockRows, &all_128);
@@ -456,6 +458,7 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
   if ((do_row && capacity_rows > 0 && row_amax == nullptr) ||
       (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
     return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(row_amax, 16) || !aligned(col_amax, 16)) return NVFP4_ERR_UNSUPPORTED;
   DeviceRouting routing;  // tiled scales need 128-row groups: checked on the device
   s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups,
                      out->scale_layout == NVFP4_SCALE_TILED_128X4 ? kRows : kBlockRows, routing);
