@@ -190,7 +190,10 @@ NVFP4RS_API nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t 
  * Grouped cast, graph-safe routing: nvfp4_group_cast with the routing of
  * nvfp4_group_amax_graphsafe (same arguments, same status rules; status_dev
  * is reset to 0 by this call too). Byte-identical to nvfp4_group_cast for
- * equal routing. One launch plus one memset of status.
+ * equal routing. One memset of status and two launches: the kernel for
+ * 128-aligned groups and the one for any groups, each of which checks the
+ * device routing and returns at once unless it is the one to run (uniform
+ * groups and tiled scales need only one).
  */
 NVFP4RS_API nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
                                         const int64_t* first_dims_dev,

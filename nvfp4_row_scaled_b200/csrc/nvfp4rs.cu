@@ -105,7 +105,7 @@ nvfp4_status device_routing(const int64_t* first_dims, const int64_t* offsets, i
     return NVFP4_ERR_INVALID_ARG;
   }
   if (!aligned(status, 4) || !aligned(first_dims, 8) || !aligned(offsets, 8)) return NVFP4_ERR_UNSUPPORTED;
-  r = DeviceRouting{first_dims, offsets, status, K, capacity_rows, E, align, m};
+  r = DeviceRouting{first_dims, offsets, status, K, capacity_rows, E, align, m, 0};
   return NVFP4_OK;
 }
 
@@ -466,7 +466,22 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK) return s;
   if (K == 0) return NVFP4_OK;
-  return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
+  if (out->scale_layout == NVFP4_SCALE_TILED_128X4)  // 128-row groups only: every tile is plain
+    return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
+                       /*general=*/false, stream);
+  if (routing.uniform_rows >= 0)
+    return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
+                       routing.uniform_rows % kRows != 0, stream);
+  // The host cannot see whether the groups are 128-aligned: enqueue the plain
+  // instantiation, which runs only if they all are, and the general one,
+  // which runs only if some are not (the other exits after the routing).
+  DeviceRouting plain = routing, general = routing;
+  plain.only_128 = 1;
+  general.only_128 = -1;
+  s = launch_cast(plain, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
+                  /*general=*/false, stream);
+  if (s != NVFP4_OK) return s;
+  return launch_cast(general, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
                      /*general=*/true, stream);
 }
 

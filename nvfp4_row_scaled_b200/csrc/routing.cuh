@@ -60,6 +60,10 @@ struct HostRouting {
 // With uniform_rows >= 0 the two arrays are absent and every group has
 // uniform_rows rows (the host checked E * uniform_rows <= capacity_rows).
 // Groups whose size is not a multiple of `align` are NVFP4_ERR_UNSUPPORTED.
+// `only_128`: +1 runs the kernel only when every group is a multiple of 128
+// rows, -1 only when some group is not, 0 always; a kernel that does not run
+// returns at once without touching the status (two instantiations of one
+// step are enqueued back to back and exactly one of them runs).
 struct DeviceRouting {
   const int64_t* first_dims;
   const int64_t* tensor_offsets;
@@ -69,6 +73,7 @@ struct DeviceRouting {
   int32_t E;
   int32_t align;
   int64_t uniform_rows;
+  int32_t only_128;
 
   __device__ __forceinline__ void load(RoutingSmem& s, int32_t* off_smem) const {
     if (uniform_rows >= 0) {
@@ -82,7 +87,7 @@ struct DeviceRouting {
       __syncthreads();
       return;
     }
-    int bad_routing = 0, bad_align = 0;
+    int bad_routing = 0, bad_align = 0, not_128 = 0;
     for (int i = threadIdx.x; i <= E; i += blockDim.x) {
       const int64_t o = tensor_offsets[i];
       if ((i == 0 && o != 0) || o < 0 || o % K != 0 || o / K > capacity_rows) {
@@ -95,15 +100,18 @@ struct DeviceRouting {
         const int64_t next = tensor_offsets[i + 1];
         if (fd < 0 || fd > capacity_rows || next - o != fd * K) bad_routing = 1;
         if (fd % align != 0) bad_align = 1;
+        if (fd % kRows != 0) not_128 = 1;
       }
     }
     bad_routing = __syncthreads_or(bad_routing);
     bad_align = __syncthreads_or(bad_align);
+    not_128 = __syncthreads_or(not_128);
     if (threadIdx.x == 0) {
       const int code = bad_routing ? NVFP4_ERR_ROUTING : (bad_align ? NVFP4_ERR_UNSUPPORTED : 0);
+      const bool skip = (only_128 > 0 && not_128) || (only_128 < 0 && !not_128);
       s.off = off_smem;
       s.E = E;
-      s.ok = code == 0;
+      s.ok = code == 0 && !skip;
       s.total = code == 0 ? off_smem[E] : 0;
       if (code != 0) *status = code;
     }
