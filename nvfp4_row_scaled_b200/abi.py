@@ -194,7 +194,9 @@ def nvfp4_group_amax_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
 def nvfp4_group_cast_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
-                               status: torch.Tensor, stream=None, scale_layout: int = NVFP4_SCALE_COMPACT, num_groups: Optional[int] = None) -> None:
+                               status: torch.Tensor, stream=None,
+                               scale_layout: int = NVFP4_SCALE_COMPACT,
+                               num_groups: Optional[int] = None) -> None:
     o = _outputs(out, scale_layout)
     rc = lib().nvfp4_group_cast_graphsafe(
         _dev(x, torch.bfloat16, "x"), x.shape[0], x.shape[1],
@@ -232,7 +234,8 @@ def nvfp4_group_quantize_graphsafe(x: torch.Tensor, first_dims: torch.Tensor,
                                    tensor_offsets: torch.Tensor, row_amax: Optional[torch.Tensor],
                                    col_amax: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
                                    workspace: torch.Tensor, status: torch.Tensor,
-                                   stream=None, scale_layout: int = NVFP4_SCALE_COMPACT, num_groups: Optional[int] = None) -> None:
+                                   stream=None, scale_layout: int = NVFP4_SCALE_COMPACT,
+                                   num_groups: Optional[int] = None) -> None:
     o = _outputs(out, scale_layout)
     wp, wb = _workspace(workspace)
     rc = lib().nvfp4_group_quantize_graphsafe(

@@ -179,3 +179,42 @@ def test_gemm_with_unit_amax_then_post_scale_matches_true_dequant():
     torch.cuda.synchronize()
     scale = y_true.abs().amax(dim=1, keepdim=True).clamp_min(1e-30)
     assert float(((y - y_true).abs() / scale).max()) < 1e-5
+
+
+def test_tiled_scales_graphsafe_cuda_graph_replays():
+    w = workloads.config4(capacity=4096)
+    x = w.x.cuda()
+    cap, K = x.shape
+    E = w.E
+    fd = torch.zeros(E, dtype=torch.int64, device="cuda")
+    offs = torch.zeros(E + 1, dtype=torch.int64, device="cuda")
+    ra, ca = abi.alloc_amax(cap, K, E)
+    out = abi.alloc_outputs(cap, K, E)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def run():
+        abi.nvfp4_group_amax_graphsafe(x, fd, offs, ra, ca, st)
+        abi.nvfp4_group_cast_graphsafe(x, fd, offs, ra, ca, out, st, scale_layout=TILED)
+
+    def set_routing(splits):
+        f, o = abi.routing_tensors(splits, K)
+        fd.copy_(f)
+        offs.copy_(o)
+
+    set_routing(w.routings[0])
+    run()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run()
+    for splits in w.routings[:4]:
+        set_routing(splits)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        total = sum(splits)
+        got = {k: v.cpu().numpy() for k, v in out.items()}
+        cut = {"row_data": total, "row_scale": total, "row_s2": total,
+               "col_data": total * K // 2, "col_scale": total * K // 16}
+        got = {k: (v[:cut[k]] if k in cut else v) for k, v in got.items()}
+        assert_identical(got, cast(w.x[:total], splits, TILED), keys=list(KEYS), what="tiled replay")

@@ -151,3 +151,36 @@ def test_full_size_deepseek_sampled_groups():
         assert np.array_equal(got["row_scale"][o:o + m], want["row_scale"])
         assert np.array_equal(got["col_data"][K * o // 2:K * (o + m) // 2], want["col_data"])
         assert np.array_equal(got["col_scale"][K * o // 32:K * (o + m) // 32], want["col_scale"])
+
+
+def test_graphsafe_cuda_graph_replays():
+    """Captured once, replayed after new routings are written to the device
+    buffers: every replay equals the host-split cast of that routing."""
+    w = workloads.config4(capacity=4096)
+    x = w.x.cuda()
+    cap, K = x.shape
+    fd = torch.zeros(w.E, dtype=torch.int64, device="cuda")
+    offs = torch.zeros(w.E + 1, dtype=torch.int64, device="cuda")
+    out = abi.alloc_mx_outputs(cap, K)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def set_routing(splits):
+        f, o = abi.routing_tensors(splits, K)
+        fd.copy_(f)
+        offs.copy_(o)
+
+    set_routing(w.routings[0])
+    abi.nvfp4_mx_group_cast_graphsafe(x, fd, offs, out, st)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        abi.nvfp4_mx_group_cast_graphsafe(x, fd, offs, out, st)
+    for splits in w.routings[:4]:
+        set_routing(splits)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        total = sum(splits)
+        got = {k: v.cpu().numpy() for k, v in out.items()}
+        cut = {"row_data": total, "row_scale": total, "col_data": total * K // 2, "col_scale": total * K // 32}
+        check({k: v[:cut[k]] for k, v in got.items()}, gpu_mx(w.x[:total], splits), "replay")
