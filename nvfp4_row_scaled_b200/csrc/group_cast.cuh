@@ -455,6 +455,36 @@ __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut&
   }
 }
 
+// A whole tile of one group that is not on the 128-row grid: colwise codes
+// as 8-byte pieces (the runs are 8-byte aligned), colwise scales as bytes.
+__device__ __forceinline__ void store_staged_single(const CastStage& st, const CastOut& out, int K, int32_t o_g,
+                                                    int64_t m_g, int32_t r0, int c0, int t, bool do_row,
+                                                    bool do_col, uint64_t keep) {
+  if (do_col) {
+    const size_t half_m = static_cast<size_t>(m_g) >> 1, m16 = static_cast<size_t>(m_g) >> 4;
+    uint8_t* gd = out.col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
+    uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++) {
+      const int u = kk * kCastThreads + t;
+      const int col = u >> 3, b = u & 7;
+      const int sw = (col >> 3) & 7;
+      st_global_u2_hint(gd + static_cast<size_t>(c0 + col) * half_m + 8 * b,
+                        *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * (b ^ sw)]), keep);
+      gs[static_cast<size_t>(c0 + col) * m16 + b] = st.col_scale[b * kCols + col];
+    }
+  }
+  if (do_row) {
+    uint32_t s0 = 0u, s1 = 0u;
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+      s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
+      s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
+    }
+    st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4), make_uint2(s0, s1), keep);
+  }
+}
+
 // (Never sees tiled scales: those need 128-aligned groups, whose tiles are
 // all plain.) Stores of a tile that store_staged cannot take: a tile crossing a group
 // boundary, the short last tile, or a group that does not start and end on
@@ -466,16 +496,16 @@ __device__ __noinline__ void store_staged_general(const CastStage& st, const Cas
                                                      const RoutingSmem& rs, int K, int32_t r0, int c0,
                                                      int t, int valid, bool mixed, int g, bool do_row,
                                                      bool do_col, uint64_t keep) {
-  if (do_col) {
+  // thread t always stores 16-row block t % 8 (of columns t / 8 + 16 kk)
+  const int b = t & 7;
+  if (do_col && kBlockRows * b < valid) {
+    const int32_t r = r0 + kBlockRows * b;
+    const int gb = mixed ? group_of_row(rs, r) : g;
+    const int32_t o = rs.off[gb];
+    const size_t m = static_cast<size_t>(rs.off[gb + 1] - o);
 #pragma unroll 2
     for (int kk = 0; kk < 8; kk++) {
-      const int u = kk * kCastThreads + t;
-      const int col = u >> 3, b = u & 7;
-      if (kBlockRows * b >= valid) continue;
-      const int32_t r = r0 + kBlockRows * b;
-      const int gb = mixed ? group_of_row(rs, r) : g;
-      const int32_t o = rs.off[gb];
-      const size_t m = static_cast<size_t>(rs.off[gb + 1] - o);
+      const int col = (kk * kCastThreads + t) >> 3;
       const int sw = (col >> 3) & 7;
       const uint2 d = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * (b ^ sw)]);
       st_global_u2_hint(out.col_data + (static_cast<size_t>(K) * o >> 1) + static_cast<size_t>(c0 + col) * (m >> 1) +
@@ -602,11 +632,17 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
         sm.col_senc[0][t] = s_enc_of(a);
         slow |= !fast_path_amax(a);
       } else {  // one column table per 16-row block, from the block's group
+        int gb = g, gprev = -1;
+        float e = 1.0f;
         for (int b = 0; kBlockRows * b < valid; b++) {
-          const int gb = group_of_row(rs, r0 + kBlockRows * b);
-          const float a = col_amax[static_cast<size_t>(gb) * K + c0 + t];
-          sm.col_senc[b][t] = s_enc_of(a);
-          slow |= !fast_path_amax(a);
+          while (rs.off[gb + 1] <= r0 + kBlockRows * b) gb++;  // groups only move forward
+          if (gb != gprev) {  // a new group (a tile holds few): its column scale
+            const float a = col_amax[static_cast<size_t>(gb) * K + c0 + t];
+            e = s_enc_of(a);
+            slow |= !fast_path_amax(a);
+            gprev = gb;
+          }
+          sm.col_senc[b][t] = e;
         }
       }
     }
@@ -651,6 +687,8 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
       const bool mixed2 = kGeneral && o_g + m_g < r0 + valid2;
       if (!kGeneral || (!mixed2 && valid2 == kRows && ((o_g | m_g) & (kRows - 1)) == 0))
         store_staged<kTiled>(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
+      else if (!mixed2 && valid2 == kRows)
+        store_staged_single(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
       else
         store_staged_general(st, out, rs, K, r0, c0, t, valid2, mixed2, g, do_row, do_col, keep);
     }
