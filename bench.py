@@ -355,7 +355,26 @@ def main():
     barrier()
     mx_ms = max_over_ranks(timed(mx_step, args.steps), world, dev)
     mx_bytes = 2 * N + 2 * (N // 2 + N // 32)
-    del mx_out
+
+    # ---- dequantize of the rowwise outputs to fp32 (NVFP4 and MXFP4)
+    step()
+    deq = torch.empty(M, K, dtype=torch.float32, device=dev)
+
+    def deq_nv():
+        abi.nvfp4_dequantize(out["row_data"], out["row_scale"], out["row_s2"], M, K, deq)
+
+    def deq_mx():
+        abi.nvfp4_mx_dequantize(mx_out["row_data"], mx_out["row_scale"], M, K, deq)
+
+    for _ in range(args.warmup):
+        deq_nv()
+        deq_mx()
+    barrier()
+    deq_nv_ms = max_over_ranks(timed(deq_nv, args.steps), world, dev)
+    deq_mx_ms = max_over_ranks(timed(deq_mx, args.steps), world, dev)
+    deq_nv_bytes = N // 2 + N // 16 + 4 * M + 4 * N
+    deq_mx_bytes = N // 2 + N // 32 + 4 * N
+    del mx_out, deq
 
     # ---- end to end through the C ABI with host buffers (pinned)
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
@@ -463,6 +482,15 @@ def main():
             "value": round(job_throughput(N, world, mx_ms), 3),
             "hbm_gbs": round(mx_bytes / (mx_ms * 1e-3) / 1e9, 1),
             "hbm_frac_of_peak": round(mx_bytes / (mx_ms * 1e-3) / 1e9 / peak, 4),
+        },
+        "dequantize": {
+            "what": "rowwise outputs [sum_M, K] -> fp32",
+            "nvfp4": {"ms": round(deq_nv_ms, 4),
+                      "hbm_gbs": round(deq_nv_bytes / (deq_nv_ms * 1e-3) / 1e9, 1),
+                      "hbm_frac_of_peak": round(deq_nv_bytes / (deq_nv_ms * 1e-3) / 1e9 / peak, 4)},
+            "mxfp4": {"ms": round(deq_mx_ms, 4),
+                      "hbm_gbs": round(deq_mx_bytes / (deq_mx_ms * 1e-3) / 1e9, 1),
+                      "hbm_frac_of_peak": round(deq_mx_bytes / (deq_mx_ms * 1e-3) / 1e9 / peak, 4)},
         },
         "gpu_launches": 2 * args.steps,
         "clocks": clk,

@@ -189,27 +189,4 @@ mx_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ 
   }
 }
 
-// MXFP4 dequantize: one thread per 32-element block (16 code bytes, 1 scale).
-constexpr int kMxDequantThreads = 256;
-
-__global__ void __launch_bounds__(kMxDequantThreads)
-mx_dequant_kernel(const uint4* __restrict__ data, const uint8_t* __restrict__ scale, int64_t blocks,
-                  float4* __restrict__ out) {
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * kMxDequantThreads + threadIdx.x; b < blocks;
-       b += static_cast<int64_t>(gridDim.x) * kMxDequantThreads) {
-    const uint4 d = data[b];
-    const uint32_t code = scale[b];  // 2^(code - 127): code 0 is the subnormal 2^-127, 0xFF is NaN
-    const float sc = code == 0u ? 0x1p-127f : (code == 0xFFu ? __uint_as_float(0x7FC00000u) : __uint_as_float(code << 23));
-    const uint32_t w[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      float f[8];
-      e2m1x8_to_f32(w[j], f);
-      out[b * 8 + 2 * j] = make_float4(__fmul_rn(f[0], sc), __fmul_rn(f[1], sc), __fmul_rn(f[2], sc), __fmul_rn(f[3], sc));
-      out[b * 8 + 2 * j + 1] =
-          make_float4(__fmul_rn(f[4], sc), __fmul_rn(f[5], sc), __fmul_rn(f[6], sc), __fmul_rn(f[7], sc));
-    }
-  }
-}
-
 }  // namespace nvfp4rs

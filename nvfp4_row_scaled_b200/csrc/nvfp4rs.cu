@@ -373,6 +373,23 @@ nvfp4_status launch_mx_cast(const Routing& routing, const void* x, int64_t rows,
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), o));
 }
 
+// One warp per row at a time, every SM filled (8 CTAs of 256 threads).
+template <bool kMx>
+nvfp4_status launch_dequant(const uint8_t* data, const uint8_t* scale, const float* s2, int64_t rows, int64_t cols,
+                            float* out_f32, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows_per_cta = kDequantThreads / 32;
+  int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kDequantThreads);
+  cfg.stream = stream;
+  return cuda_status(cudaLaunchKernelEx(&cfg, dequant_kernel<kMx>, reinterpret_cast<const uint16_t*>(data), scale, s2,
+                                        rows, cols, reinterpret_cast<float4*>(out_f32)));
+}
+
 }  // namespace
 
 extern "C" {
@@ -492,20 +509,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const f
   if (data == nullptr || scale == nullptr || s2 == nullptr || out_f32 == nullptr)
     return NVFP4_ERR_INVALID_ARG;
   if (!aligned(data, 8) || !aligned(out_f32, 16) || !aligned(s2, 4)) return NVFP4_ERR_UNSUPPORTED;
-  const int64_t bpr = cols / 16;
-  const int64_t n = rows * bpr;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t grid = (n + kDequantThreads - 1) / kDequantThreads;
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
-  if (grid > cap) grid = cap;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kDequantThreads);
-  cfg.stream = stream;
-  return cuda_status(cudaLaunchKernelEx(&cfg, dequant_kernel, reinterpret_cast<const uint2*>(data),
-                                        scale, s2, rows, bpr, reinterpret_cast<float4*>(out_f32)));
+  return launch_dequant<false>(data, scale, s2, rows, cols, out_f32, stream);
 }
 
 size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, int32_t num_groups) {
@@ -660,17 +664,7 @@ nvfp4_status nvfp4_mx_dequantize(const uint8_t* data, const uint8_t* scale, int6
   if (rows == 0 || cols == 0) return NVFP4_OK;
   if (data == nullptr || scale == nullptr || out_f32 == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(data, 16) || !aligned(out_f32, 16)) return NVFP4_ERR_UNSUPPORTED;
-  const int64_t blocks = rows * (cols / 32);
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t grid = (blocks + kMxDequantThreads - 1) / kMxDequantThreads;
-  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kMxDequantThreads);
-  cfg.stream = stream;
-  return cuda_status(cudaLaunchKernelEx(&cfg, mx_dequant_kernel, reinterpret_cast<const uint4*>(data), scale, blocks,
-                                        reinterpret_cast<float4*>(out_f32)));
+  return launch_dequant<true>(data, scale, nullptr, rows, cols, out_f32, stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status status) {
