@@ -408,8 +408,8 @@ def main():
     dom_ms = cast_ms if dominant == "cast" else amax_ms
     achieved = b[dominant] / (dom_ms * 1e-3) / 1e9
     workload_name = w.name
-    traffic = traffic_record("group_cast_kernel" if dominant == "cast" else "group_amax_kernel",
-                             workload_name)
+    dom_kernel = "group_cast_plain_kernel" if dominant == "cast" else "group_amax_kernel"
+    traffic = traffic_record(dom_kernel, workload_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(w)
@@ -439,7 +439,7 @@ def main():
         "hbm_frac_of_peak": round(b["step"] / (ms_per_step * 1e-3) / 1e9 / peak, 4),
         "kernels_ms": {"amax": round(amax_ms, 4), "cast": round(cast_ms, 4)},
         "roofline": {
-            "kernel": f"group_{dominant}_kernel",
+            "kernel": dom_kernel,
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,

@@ -8,7 +8,12 @@
 // scaling; TransformerEngine #3324 (row-scaled backward for GroupedLinear,
 // summary) adds the columnwise (transposed) operand with per-column amax.
 //
-// Structure (sm_100a):
+// This file holds what both cast kernels share (TMA and mbarrier helpers,
+// the lane patch, encode_patch, the scale stores) and the general kernel for
+// groups that are multiples of 16 rows anywhere; the kernel for groups on the
+// 128-row grid is in group_cast_plain.cuh.
+//
+// Structure of the general kernel (sm_100a):
 //  - Persistent CTAs (three per SM), each taking every gridDim-th 128 x 128
 //    tile of x in row-major tile order, so CTAs running at the same time read
 //    neighbouring tiles of the same rows. Group sizes are multiples of 16, so
@@ -29,8 +34,8 @@
 //    table of every E4M3 value and its correctly rounded reciprocal, and
 //    Markstein's correction (codec.cuh).
 //  - Outputs that are not contiguous per lane (colwise data and scales,
-//    rowwise scales) are staged in shared memory and stored as full 16- or
-//    8-byte pieces of contiguous runs, with an L2 evict-last hint: a group's
+//    rowwise scales) are staged in shared memory and stored as full 8- or
+//    16-byte pieces of contiguous runs, with an L2 evict-last hint: a group's
 //    transposed outputs and the 8-byte scale pieces fill their sectors from
 //    several tiles, and should meet in L2 before being written back.
 // Tiles of groups that are not multiples of 128 rows, mixed tiles and the
@@ -77,9 +82,6 @@ struct CastSmem {
   float2 e4m3[128];                   // {value, RN(1/value)} per E4M3 code
   float row_senc[kRows];
   float col_senc[kRows / kBlockRows][kCols];  // per 16-row block: [0] only, unless the tile is mixed
-  float pf_col[kStages][kCols];  // plain kernel: the stage's tile's column amax (bulk copy)
-  float pf_row[kStages][kRows];  // its row amax, when it starts a new row tile for this CTA
-  int pf_g[kStages];             // its group
   uint64_t full[kStages];
 };
 
@@ -177,26 +179,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Plain cast kernel: tile `tl` into stage s together with what its encode
-// scales need -- its group, the 128 column amax of that group and, when the
-// tile starts a new row tile for this CTA, the 128 row amax -- by bulk copies
-// completing on the tile's own mbarrier, so the values arrive with the tile
-// (thread 0 only; amax pointers NULL for a direction not requested).
-__device__ __forceinline__ void issue_tile_amax(CastSmem& sm, const CUtensorMap* map, int s, int tl, int n_ct,
-                                                const RoutingSmem& rs, int K, const float* row_amax,
-                                                const float* col_amax, bool new_row) {
-  const int rt = tl / n_ct, ct = tl - rt * n_ct;
-  const int g = group_of_row(rs, rt * kRows);
-  sm.pf_g[s] = g;
-  const bool rows = row_amax != nullptr && new_row;
-  mbar_expect_tx(&sm.full[s], kTileBytes + (col_amax != nullptr ? 512u : 0u) + (rows ? 512u : 0u));
-  const uint64_t pol = policy_evict_first();
-  tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s], pol);
-  tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s], pol);
-  if (col_amax != nullptr) bulk_load(sm.pf_col[s], col_amax + static_cast<size_t>(g) * K + ct * kCols, 512u, &sm.full[s]);
-  if (rows) bulk_load(sm.pf_row[s], row_amax + static_cast<size_t>(rt) * kRows, 512u, &sm.full[s]);
-}
-
 // Tile number `tl` of the row-major tile order (read once: evict first).
 __device__ __forceinline__ void issue_tile(CastSmem& sm, const CUtensorMap* map, int s, int tl,
                                            int n_ct) {
@@ -218,21 +200,16 @@ __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
   *reinterpret_cast<uint32_t*>(p) = v;
 }
 
-// Everything one lane does for one tile after its 16 x 8 patch is in
-// registers: block scales of both directions, all codes, the rowwise data
-// stores and the staging of the other outputs. kExact selects the
-// IEEE-divide block scales (tiles with a row or column amax outside the
-// shortcut's range).
 // The codes of a lane's 16 x 8 patch, once the multipliers are known: renc[i]
 // multiplies row i (rowwise codes, stored straight to rdst + i * row_pitch
-// when row_store), cenc2[q] the column pair (2q, 2q+1) (colwise codes, staged
-// transposed in st.col_data: 8 bytes per column at slot rb ^ (cc % 8)). Shared
-// by the NVFP4 and the MXFP4 casts.
+// when row_store), cenc2[q] the column pair (2q, 2q+1) (colwise codes, handed
+// to col_sink(half, cw): cw[q] holds rows 8*half .. 8*half+7 of column q, row
+// 8*half in the low nibble). Shared by the NVFP4 and the MXFP4 casts.
+template <class ColSink>
 __device__ __forceinline__ void encode_codes(const uint4 (&v)[16], const float (&renc)[16],
-                                             const uint64_t (&cenc2)[4], CastStage& st, bool do_row,
-                                             bool do_col, int cc, int rb, uint8_t* rdst, size_t row_pitch,
-                                             bool row_store) {
-  const int slot = rb ^ (cc & 7);
+                                             const uint64_t (&cenc2)[4], bool do_row, bool do_col,
+                                             uint8_t* rdst, size_t row_pitch, bool row_store,
+                                             ColSink&& col_sink) {
 #pragma unroll
   for (int half = 0; half < 2; half++) {
     uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
@@ -279,12 +256,23 @@ __device__ __forceinline__ void encode_codes(const uint4 (&v)[16], const float (
       cw[5] = prmt(u0, u2, 0x7632);
       cw[6] = prmt(u1, u3, 0x5410);
       cw[7] = prmt(u1, u3, 0x7632);
-#pragma unroll
-      for (int q = 0; q < 8; q++)
-        *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
+      col_sink(half, cw);
     }
   }
 }
+
+// The staging sink of encode_codes: the column words of lane (cc, rb) go to
+// st.col_data, 8 bytes per column at slot rb ^ (cc % 8).
+struct StageColSink {
+  CastStage& st;
+  int cc, rb;
+  __device__ __forceinline__ void operator()(int half, const uint32_t (&cw)[8]) const {
+    const int slot = rb ^ (cc & 7);
+#pragma unroll
+    for (int q = 0; q < 8; q++)
+      *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
+  }
+};
 
 // The shared tables a tile's encode reads: {value, RN(1/value)} of every
 // E4M3 code, and S_enc of the tile's 128 rows and 128 columns.
@@ -294,10 +282,17 @@ struct EncodeTables {
   const float* col_senc;
 };
 
-template <bool kExact>
-__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, CastStage& st,
-                                             bool do_row, bool do_col, int cc, int rb,
-                                             uint8_t* rdst, size_t row_pitch, bool row_store = true) {
+// Everything one lane does for one tile after its 16 x 8 patch is in
+// registers: block scales of both directions, all codes, the rowwise data
+// stores, the staging of the block scales (col_stg: [row block][column],
+// row_stg: [column block][row], both 128 wide) and the colwise codes handed
+// to col_sink. cc (0..15) is the lane's 8-column chunk of the tile, rb (0..7)
+// its 16-row block. kExact selects the IEEE-divide block scales (tiles with a
+// row or column amax outside the shortcut's range).
+template <bool kExact, class ColSink>
+__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, uint8_t* col_stg,
+                                             uint8_t* row_stg, bool do_row, bool do_col, int cc, int rb,
+                                             uint8_t* rdst, size_t row_pitch, bool row_store, ColSink&& col_sink) {
   const int rl = 16 * rb;
   const bool odd = cc & 1;
 
@@ -324,7 +319,7 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
       cenc2[q] = pack2(e0, e1);
       s8w[q >> 1] |= p2 << (16 * (q & 1));
     }
-    *reinterpret_cast<uint2*>(&st.col_scale[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
+    *reinterpret_cast<uint2*>(&col_stg[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
   }
 
   // ------------------------------------------------------ rowwise scales
@@ -359,13 +354,22 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
     const uint32_t so0 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[0], 1);
     const uint32_t so1 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[1], 1);
     if (!odd) {
-      *reinterpret_cast<uint4*>(&st.row_scale[(cc >> 1) * kRows + rl]) =
+      *reinterpret_cast<uint4*>(&row_stg[(cc >> 1) * kRows + rl]) =
           make_uint4(s8mine[0], s8mine[1], so0, so1);
     }
   }
 
   // -------------------------------------------------------------- codes
-  encode_codes(v, renc, cenc2, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
+  encode_codes(v, renc, cenc2, do_row, do_col, rdst, row_pitch, row_store, col_sink);
+}
+
+// encode_patch with every output but the rowwise data staged in st.
+template <bool kExact>
+__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, CastStage& st,
+                                             bool do_row, bool do_col, int cc, int rb,
+                                             uint8_t* rdst, size_t row_pitch, bool row_store = true) {
+  encode_patch<kExact>(v, tab, st.col_scale, st.row_scale, do_row, do_col, cc, rb, rdst, row_pitch, row_store,
+                       StageColSink{st, cc, rb});
 }
 
 // The 128x4-tiled scale layout (the grouped GEMM's swizzle contract; see the
@@ -388,9 +392,6 @@ __device__ __forceinline__ uint2 tiled_piece(const uint8_t* stg, int t) {
   return make_uint2(w[0], w[1]);
 }
 
-// Stores of the outputs a tile staged: colwise data (64 bytes per column,
-// four 16-byte pieces), colwise scales (8 bytes per column) and rowwise scales
-// (8 bytes per row), all with the L2 evict-last policy `keep`.
 // The staged colwise codes of a whole tile of a 128-aligned group: 64 bytes
 // per column (four 16-byte pieces) into the group's transposed slice.
 __device__ __forceinline__ void store_col_data(const CastStage& st, uint8_t* col_data, int K, int32_t o_g,
@@ -409,12 +410,15 @@ __device__ __forceinline__ void store_col_data(const CastStage& st, uint8_t* col
   }
 }
 
+// The staged block scales of a tile of a 128-aligned group: colwise
+// (col_stg [row block][column]) 8 bytes per column, rowwise (row_stg
+// [column block][row]) 8 bytes per row, compact or as two whole 128x4 tiles
+// per direction (kTiled).
 template <bool kTiled>
-__device__ __forceinline__ void store_staged(const CastStage& st, const CastOut& out, int K,
-                                             int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
+__device__ __forceinline__ void store_scales(const uint8_t* col_stg, const uint8_t* row_stg, const CastOut& out,
+                                             int K, int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
                                              bool do_row, bool do_col, uint64_t keep) {
   if (do_col) {
-    store_col_data(st, out.col_data, K, o_g, m_g, r0, c0, t, keep);
     if (kTiled) {
       // the tile's 128 x 8 block scales are two whole 128x4 tiles of the
       // group's [K, m_g/16] scale matrix: tile row c0/128, tile columns
@@ -422,15 +426,15 @@ __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut&
       const int j = t >> 6;
       uint8_t* blk = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) +
                      ((static_cast<size_t>(c0 >> 7) * (static_cast<size_t>(m_g) >> 6)) + ((r0 - o_g) >> 6) + j) * 512;
-      st_global_u2_hint(blk + tiled_piece_offset(t), tiled_piece(st.col_scale + 4 * j * kCols, t), keep);
+      st_global_u2_hint(blk + tiled_piece_offset(t), tiled_piece(col_stg + 4 * j * kCols, t), keep);
     } else {
       const size_t m16 = static_cast<size_t>(m_g) >> 4;
       uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
       uint32_t s0 = 0u, s1 = 0u;
 #pragma unroll
       for (int r = 0; r < 4; r++) {
-        s0 |= static_cast<uint32_t>(st.col_scale[r * kCols + t]) << (8 * r);
-        s1 |= static_cast<uint32_t>(st.col_scale[(r + 4) * kCols + t]) << (8 * r);
+        s0 |= static_cast<uint32_t>(col_stg[r * kCols + t]) << (8 * r);
+        s1 |= static_cast<uint32_t>(col_stg[(r + 4) * kCols + t]) << (8 * r);
       }
       st_global_u2_hint(gs + static_cast<size_t>(c0 + t) * m16, make_uint2(s0, s1), keep);
     }
@@ -441,18 +445,28 @@ __device__ __forceinline__ void store_staged(const CastStage& st, const CastOut&
       // r0/128, tile columns c0/64 + 0, 1 (K/64 tiles per tile row)
       const int j = t >> 6;
       uint8_t* blk = out.row_scale + (static_cast<size_t>(r0 >> 7) * (K >> 6) + (c0 >> 6) + j) * 512;
-      st_global_u2_hint(blk + tiled_piece_offset(t), tiled_piece(st.row_scale + 4 * j * kRows, t), keep);
+      st_global_u2_hint(blk + tiled_piece_offset(t), tiled_piece(row_stg + 4 * j * kRows, t), keep);
     } else {
       uint32_t s0 = 0u, s1 = 0u;
 #pragma unroll
       for (int r = 0; r < 4; r++) {
-        s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
-        s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
+        s0 |= static_cast<uint32_t>(row_stg[r * kRows + t]) << (8 * r);
+        s1 |= static_cast<uint32_t>(row_stg[(r + 4) * kRows + t]) << (8 * r);
       }
       st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
                         make_uint2(s0, s1), keep);
     }
   }
+}
+
+// Everything a tile of a 128-aligned group staged in st: colwise data, then
+// the block scales.
+template <bool kTiled>
+__device__ __forceinline__ void store_staged(const CastStage& st, const CastOut& out, int K,
+                                             int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
+                                             bool do_row, bool do_col, uint64_t keep) {
+  if (do_col) store_col_data(st, out.col_data, K, o_g, m_g, r0, c0, t, keep);
+  store_scales<kTiled>(st.col_scale, st.row_scale, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
 }
 
 // A whole tile of one group that is not on the 128-row grid: colwise codes
@@ -529,11 +543,11 @@ __device__ __noinline__ void store_staged_general(const CastStage& st, const Cas
 
 // ------------------------------------------------------------------ kernel
 
-// kGeneral = false: every group is a multiple of 128 rows starting on a
-// 128-row boundary (the host or the device routing checked), so every tile
-// is plain and the general-tile code is compiled out. kTiled: both scale
-// outputs in the 128x4-tiled layout (only with kGeneral = false).
-template <class Routing, bool kGeneral, bool kTiled>
+// The general cast: groups that are multiples of 16 rows anywhere (the
+// 128-aligned case runs group_cast_plain_kernel). A tile may cross group
+// boundaries (mixed: one column-scale table per 16-row block) and the last
+// row tile may be short.
+template <class Routing>
 __global__ void __launch_bounds__(kCastThreads, 3)
 group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
                   int32_t K, const float* __restrict__ row_amax,
@@ -564,7 +578,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
   }
   sm.e4m3[t] = e4m3_entry(t);
 
-  // this CTA's tiles: a contiguous range of the row-major tile order
+  // this CTA's tiles: every gridDim-th of the row-major tile order
   const int n_ct = K >> 7;
   const int n_tiles = ((rs.total + kRows - 1) >> 7) * n_ct;  // the last row tile may be short
   const int G = gridDim.x;
@@ -575,15 +589,8 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     slow_tile[1] = 0;
   }
   __syncthreads();
-  if (t == 0) {
-    for (int s = 0; s < kStages && blockIdx.x + s * G < n_tiles; s++) {
-      const int tl = blockIdx.x + s * G;
-      if (kGeneral)
-        issue_tile(sm, &tmap, s, tl, n_ct);
-      else
-        issue_tile_amax(sm, &tmap, s, tl, n_ct, rs, K, do_row ? row_amax : nullptr, do_col ? col_amax : nullptr, s == 0 || (tl - G) / n_ct != tl / n_ct);
-    }
-  }
+  if (t == 0)
+    for (int s = 0; s < kStages && blockIdx.x + s * G < n_tiles; s++) issue_tile(sm, &tmap, s, blockIdx.x + s * G, n_ct);
 
   const int lane = t & 31, warp = t >> 5;
   const int cc = lane & 15, h = lane >> 4;
@@ -607,28 +614,25 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     const int c0 = ct * kCols;
     if (t == 0) slow_tile[(k + 1) & 1] = 0;  // flag of the next tile (last read a tile ago)
     bool slow = false;
-    const int valid = kGeneral ? min(kRows, rs.total - r0) : kRows;  // routed rows (a multiple of 16)
-    // plain kernel: the tile's amax values come with it (issue_tile_amax)
-    bool ok = true;
-    if (!kGeneral) ok = mbar_wait(&sm.full[s], phase);
+    const int valid = min(kRows, rs.total - r0);  // routed rows (a multiple of 16)
     if (rt != cur_rt) {  // new row tile: its group(s) and its rows' encode scales
       cur_rt = rt;
-      g = kGeneral ? group_of_row(rs, r0) : sm.pf_g[s];
+      g = group_of_row(rs, r0);
       o_g = rs.off[g];
       m_g = rs.off[g + 1] - o_g;
       if (do_row) {
         const bool in = t < valid;
-        const float a = in ? (kGeneral ? row_amax[r0 + t] : sm.pf_row[s][t]) : 0.0f;
+        const float a = in ? row_amax[r0 + t] : 0.0f;
         sm.row_senc[t] = s_enc_of(a);
         row_slow = in && !fast_path_amax(a);
-        if (ct == 0 && in && ok) out.row_s2[r0 + t] = s_dec_of(a);
+        if (ct == 0 && in) out.row_s2[r0 + t] = s_dec_of(a);
       }
     }
     slow |= row_slow;
-    const bool mixed = kGeneral && o_g + m_g < r0 + valid;  // the tile crosses a group boundary
+    const bool mixed = o_g + m_g < r0 + valid;  // the tile crosses a group boundary
     if (do_col) {
       if (!mixed) {
-        const float a = kGeneral ? col_amax[static_cast<size_t>(g) * K + c0 + t] : sm.pf_col[s][t];
+        const float a = col_amax[static_cast<size_t>(g) * K + c0 + t];
         sm.col_senc[0][t] = s_enc_of(a);
         slow |= !fast_path_amax(a);
       } else {  // one column table per 16-row block, from the block's group
@@ -649,7 +653,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     if (slow) slow_tile[k & 1] = 1;
 
     // this lane's 16 x 8 patch from the swizzled stage
-    if (kGeneral) ok = mbar_wait(&sm.full[s], phase);
+    const bool ok = mbar_wait(&sm.full[s], phase);
     uint4 v[16];
     load_patch(sm.tile[s], cc, rl, v);
     if (__syncthreads_or(!ok)) {
@@ -660,11 +664,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     // this barrier: refill it with tile k+1 (tiles 0 and 1 came in the prologue).
     if (t == 0 && k >= 1 && tl + G < n_tiles) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if (kGeneral)
-        issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
-      else
-        issue_tile_amax(sm, &tmap, (k + 1) % kStages, tl + G, n_ct, rs, K, do_row ? row_amax : nullptr, do_col ? col_amax : nullptr,
-                        (tl + G) / n_ct != rt);
+      issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
     }
     // stage s is free once every thread holds its patch: it stages the outputs
     CastStage& st = *reinterpret_cast<CastStage*>(sm.tile[s]);
@@ -672,7 +672,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
                            : nullptr;
     const EncodeTables tab{sm.e4m3, sm.row_senc, sm.col_senc[mixed ? rb : 0]};
-    const bool row_store = !kGeneral || kBlockRows * rb < valid;  // false past the routed rows
+    const bool row_store = kBlockRows * rb < valid;  // false past the routed rows
     if (slow_tile[k & 1])
       encode_patch<true>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
     else
@@ -681,12 +681,13 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     // (the tile's shape again, rather than kept live through the encode) A
     // whole tile of a group that starts and ends on 128-row boundaries takes
     // store_staged, whose 16-byte colwise data and 8-byte colwise scale stores
-    // need those boundaries; every other tile, store_staged_general.
+    // need those boundaries; a whole tile of one group otherwise,
+    // store_staged_single; every other tile, store_staged_general.
     {
-      const int valid2 = kGeneral ? min(kRows, rs.total - r0) : kRows;
-      const bool mixed2 = kGeneral && o_g + m_g < r0 + valid2;
-      if (!kGeneral || (!mixed2 && valid2 == kRows && ((o_g | m_g) & (kRows - 1)) == 0))
-        store_staged<kTiled>(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
+      const int valid2 = min(kRows, rs.total - r0);
+      const bool mixed2 = o_g + m_g < r0 + valid2;
+      if (!mixed2 && valid2 == kRows && ((o_g | m_g) & (kRows - 1)) == 0)
+        store_staged<false>(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
       else if (!mixed2 && valid2 == kRows)
         store_staged_single(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
       else

@@ -87,7 +87,7 @@ __device__ __forceinline__ void mx_encode_patch(const uint4 (&v)[16], CastStage&
 #pragma unroll
     for (int i = 0; i < 16; i++) rmul[i] = 0.0f;
   }
-  encode_codes(v, rmul, cmul2, st, do_row, do_col, cc, rb, rdst, row_pitch, true);
+  encode_codes(v, rmul, cmul2, do_row, do_col, rdst, row_pitch, true, StageColSink{st, cc, rb});
 }
 
 // Outputs of the MXFP4 cast (device pointers; a direction with both NULL is skipped).

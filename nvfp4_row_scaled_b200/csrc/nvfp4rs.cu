@@ -21,6 +21,7 @@
 #include "routing.cuh"
 #include "group_amax.cuh"
 #include "group_cast.cuh"
+#include "group_cast_plain.cuh"
 #include "group_quantize.cuh"
 #include "dequant.cuh"
 #include "post_scale.cuh"
@@ -201,28 +202,33 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
   CUtensorMap map;
   if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
   // tiled scales come with 128-row groups only (checked on the host, or on
-  // the device by the routing), so their tiles are all plain
+  // the device by the routing): those run the plain kernel
   const bool tiled = out->scale_layout == NVFP4_SCALE_TILED_128X4;
-  auto kernel = tiled ? group_cast_kernel<Routing, false, true>
-                      : (general ? group_cast_kernel<Routing, true, false> : group_cast_kernel<Routing, false, false>);
-  const size_t smem = cast_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
+  // the plain kernel: one CTA per SM, three warp groups; the general one:
+  // as many 4-warp CTAs as fit
+  auto kernel = general ? group_cast_kernel<Routing>
+                        : (tiled ? group_cast_plain_kernel<Routing, true> : group_cast_plain_kernel<Routing, false>);
+  const int threads = general ? kCastThreads : kPThreads;
+  const int64_t units = general ? tiles : (tiles + kPGroups - 1) / kPGroups;
+  // + room to align the block to 1024 bytes
+  const size_t smem = (general ? cast_smem_bytes(E) : plain_smem_bytes(E)) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCastThreads, smem) != cudaSuccess)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess)
     return NVFP4_ERR_CUDA;
   if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
-  if (tiles > 0 && tiles < grid) grid = tiles;
+  if (units > 0 && units < grid) grid = units;
   if (grid < 1) grid = 1;
   CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2,
             out->scale_layout == NVFP4_SCALE_TILED_128X4};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kCastThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), row_amax,
