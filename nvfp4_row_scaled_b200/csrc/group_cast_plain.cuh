@@ -99,7 +99,7 @@ struct DirectColSink {
   }
 };
 
-// Group leader: tile `tl` (the group's k-th) into stage s, with its group's
+// One thread of the group: tile `tl` (the group's k-th) into stage s, with its group's
 // row range and the 128 column and 128 row amax it needs (NULL: direction
 // not requested), all completing on the stage's mbarrier.
 __device__ __forceinline__ void plain_issue(PlainGroup& pg, uint8_t* stage, const CUtensorMap* map, int s,
@@ -138,12 +138,6 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
   const int t = threadIdx.x;
   const bool do_row = out.row_s2 != nullptr;
   const bool do_col = out.col_s2 != nullptr;
-  if (do_col) {  // decode scales of all columns of all groups, spread over the grid
-    const int64_t n = static_cast<int64_t>(rs.E) * K;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kPThreads + t; i < n;
-         i += static_cast<int64_t>(gridDim.x) * kPThreads)
-      out.col_s2[i] = s_dec_of(col_amax[i]);
-  }
   if (t < 128) sm.e4m3[t] = e4m3_entry(t);
 
   const int j = t / kCastThreads;  // warp group
@@ -164,6 +158,13 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
   if (gt == 0)
     for (int k = 0; k < kStages && first + k * G < n_tiles; k++)
       plain_issue(pg, sm.tile[j][k], &tmap, k, k, first + k * G, n_ct, rs, K, ra, ca);
+  if (do_col) {  // decode scales of all columns of all groups, spread over the grid, while the first tiles load
+    const int64_t n = static_cast<int64_t>(rs.E) * K;
+#pragma unroll 4
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kPThreads + t; i < n;
+         i += static_cast<int64_t>(gridDim.x) * kPThreads)
+      out.col_s2[i] = s_dec_of(col_amax[i]);
+  }
 
   const int lane = gt & 31, w = gt >> 5;
   const int cc = 8 * (w & 1) + (lane & 7);  // 8-column chunk of the tile, 0..15
@@ -207,8 +208,11 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
       failed = true;
       break;
     }
-    // every patch of tile k is in registers: its stage takes tile k+2
-    if (gt == 0 && tl + 2 * G < n_tiles) {
+    // every patch of tile k is in registers: its stage takes tile k+2. The
+    // issuing thread is lane 0 of warp k % 4, so that the issue work (group
+    // search, expect_tx, four copies) does not always delay the same warp at
+    // the next barrier.
+    if (gt == 32 * (k & 3) && tl + 2 * G < n_tiles) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       plain_issue(pg, sm.tile[j][s], &tmap, s, k + 2, tl + 2 * G, n_ct, rs, K, ra, ca);
     }
