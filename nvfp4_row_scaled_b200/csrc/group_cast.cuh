@@ -662,7 +662,9 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     }
     // The other stage held tile k-1, whose staged outputs were stored before
     // this barrier: refill it with tile k+1 (tiles 0 and 1 came in the prologue).
-    if (t == 0 && k >= 1 && tl + G < n_tiles) {
+    // (issued by lane 0 of warp k % 4, so that the issue work does not always
+    // delay the same warp at the next barrier)
+    if (t == 32 * (k & 3) && k >= 1 && tl + G < n_tiles) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
     }
