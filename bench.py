@@ -376,24 +376,56 @@ def main():
     deq_mx_bytes = N // 2 + N // 32 + 4 * N
     del mx_out, deq
 
-    # ---- end to end through the C ABI with host buffers (pinned)
-    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+    # ---- end to end through the C ABI with host buffers (pinned): every step
+    # uploads its input from pinned host memory, runs the two calls and reads
+    # all its outputs back. Two device buffer sets on three streams let step
+    # i+1's upload run while step i's outputs come back (PCIe is full duplex);
+    # a buffer set is reused only after its previous step's download ended.
     e2e_steps = max(3, min(args.steps, 5))
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+    xs = [x, torch.empty_like(x)]
+    outs = [out, abi.alloc_outputs(M, K, E, dev)]
+    amaxs = [(ra, ca), abi.alloc_amax(M, K, E, dev)]
+    s_up, s_run, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    drained = [torch.cuda.Event() for _ in range(2)]
     step()
     torch.cuda.synchronize(dev)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(x_host, non_blocking=True)
-        step()
-        for k, v in out.items():
-            host_out[k].copy_(v, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_up)
+    s_run.wait_event(e0)
+    s_down.wait_event(e0)
+    for i in range(e2e_steps):
+        bi = i % 2
+        if i >= 2:
+            s_up.wait_event(computed[bi])  # step i-2 has read this input buffer
+        with torch.cuda.stream(s_up):
+            xs[bi].copy_(x_host, non_blocking=True)
+        loaded[bi].record(s_up)
+        s_run.wait_event(loaded[bi])
+        if i >= 2:
+            s_run.wait_event(drained[bi])  # step i-2's outputs are on the host
+        abi.nvfp4_group_amax(xs[bi], splits, amaxs[bi][0], amaxs[bi][1], stream=s_run)
+        abi.nvfp4_group_cast(xs[bi], splits, amaxs[bi][0], amaxs[bi][1], outs[bi], stream=s_run)
+        computed[bi].record(s_run)
+        s_down.wait_event(computed[bi])
+        with torch.cuda.stream(s_down):
+            for k, v in outs[bi].items():
+                host_out[k].copy_(v, non_blocking=True)
+        drained[bi].record(s_down)
+    s_down.wait_stream(s_up)
+    e1.record(s_down)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    # the downloaded bytes of the last step are the device's
+    for k, v in outs[(e2e_steps - 1) % 2].items():
+        if not torch.equal(host_out[k], v.cpu()):
+            raise RuntimeError(f"end-to-end download of {k} does not match the device")
+    del xs, outs, amaxs
 
     if world > 1:
         dist.destroy_process_group()
