@@ -235,9 +235,13 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
                                         col_amax, o));
 }
 
-// Persistent grid of the one-launch kernel: every CTA that fits, at most one
-// per item. The schedule's lag covers the items a CTA holds at a time: one
-// per stage of its tile ring plus the next claim.
+// Persistent grid of the one-launch kernel: one CTA per SM (three compute
+// groups each), fewer for a problem with fewer items. The schedule's lag --
+// claims between a group's last A item and its first B item -- is a few
+// rounds of every compute group in the grid, so that the A items are
+// published by the time the B items are claimed.
+constexpr int kQuantLagRounds = 3;
+
 template <class Routing>
 nvfp4_status launch_quantize(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
                              uint32_t* ws, float* row_acc, float* row_amax, float* col_amax,
@@ -260,9 +264,10 @@ nvfp4_status launch_quantize(const Routing& routing, const void* x, int64_t rows
     return NVFP4_ERR_CUDA;
   if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
-  if (tiles > 0 && 2 * tiles < grid) grid = 2 * tiles;
+  const int64_t need = (2 * tiles + kQGroups - 1) / kQGroups;  // CTAs that get an item
+  if (need < grid) grid = need;
   if (grid < 1) grid = 1;
-  const int32_t lag = static_cast<int32_t>((kQStages + 1) * grid);
+  const int32_t lag = static_cast<int32_t>(kQuantLagRounds * kQGroups * grid);
   CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2,
             out->scale_layout == NVFP4_SCALE_TILED_128X4};
   cudaLaunchConfig_t cfg = {};
