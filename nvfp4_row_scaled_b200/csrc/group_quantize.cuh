@@ -55,7 +55,7 @@
 // Publishing an A item: each compute thread arrives on the group's adone
 // barrier after its atomics (release, CTA scope); the publisher, having seen
 // the phase complete (acquire), fences (acq_rel, GPU scope) and adds one to
-// the group's done counter. The producer waits for a group with acquire
+// the group's done counter (one fence for all the items a sweep finds). The producer waits for a group with acquire
 // loads of that counter, then a proxy fence orders the TMA unit's reads of
 // the maxima after them. adone has two slots per compute group, and a slot
 // is reused only after the publisher acknowledged its previous use (aack), so
@@ -77,7 +77,7 @@ constexpr int kBItem = 1 << 30;             // item tag: B (cast); tile index be
 constexpr int kNoItem = -1;                 // the end of the sequence
 constexpr int kAbortItem = -2;              // the producer gave up on this item
 constexpr uint32_t kDoneSpinLimit = 1u << 20;  // bounded dependency waits (~1 s)
-constexpr uint32_t kIdleLimit = 1u << 22;      // idle control loops (~100 ns each) before giving up
+constexpr uint32_t kIdleLimit = 1u << 22;      // idle control loops (>= 100 ns each) before giving up
 
 // Words of the workspace before the row accumulators (a multiple of 64).
 constexpr int64_t quant_ws_header_words(int64_t E) { return (kWsDone + E + 63) / 64 * 64; }
@@ -92,15 +92,6 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
-}
-
-// Publish the finished atomics of an A item (ordered before this thread by
-// the adone barrier) and count one finished A item of the group.
-__device__ __forceinline__ void release_add_one(uint32_t* p) {
-  asm volatile(
-      "fence.acq_rel.gpu;\n\t"
-      "red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(p)
-      : "memory");
 }
 
 __device__ __forceinline__ void raise_abort(uint32_t* abort_word) { atomicExch(abort_word, 1u); }
@@ -128,7 +119,7 @@ __device__ __forceinline__ bool wait_group(const uint32_t* done, uint32_t need, 
   for (uint32_t i = 0; i < kDoneSpinLimit; i++) {
     if (ld_acquire_u32(done) >= need) return true;
     if (ld_relaxed_u32(abort_word) != 0u) return false;
-    __nanosleep(32);
+    __nanosleep(128);
   }
   return false;
 }
@@ -303,34 +294,46 @@ __device__ __forceinline__ void quantize_producer(QuantSmem& sm, int j, const Ro
 }
 
 // The publisher: publishes every A item of every compute group in the
-// group's order, and acknowledges it so the group may reuse the slot.
+// group's order, and acknowledges it so the group may reuse the slot. A
+// GPU-scope fence waits for the SM's outstanding stores (about a
+// microsecond while the compute groups stream their outputs), so one fence
+// serves every A item found ready in a sweep over the groups.
 __device__ __forceinline__ void quantize_publisher(QuantSmem& sm, uint32_t* ws) {
   uint32_t* const abort_word = ws + 1;
   uint32_t* const done = ws + kWsDone;
   int a_pub[kQGroups] = {0, 0, 0};
   uint32_t idle = 0;
   for (;;) {
-    bool progress = false, all = true;
+    bool ready[kQGroups];
+    bool any = false, all = true;
     for (int j = 0; j < kQGroups; j++) {
-      QuantGroup& pg = sm.grp[j];
       const int a = a_pub[j];
-      if (mbar_test(&pg.adone[a & 1], (a >> 1) & 1)) {
+      ready[j] = mbar_test(&sm.grp[j].adone[a & 1], (a >> 1) & 1);
+      any |= ready[j];
+    }
+    if (any) {
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+      for (int j = 0; j < kQGroups; j++) {
+        if (!ready[j]) continue;
+        QuantGroup& pg = sm.grp[j];
+        const int a = a_pub[j];
         const int g = reinterpret_cast<volatile int32_t*>(pg.pub_grp)[a & 3];
-        release_add_one(&done[g]);
+        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(&done[g]) : "memory");
         mbar_arrive(&pg.aack[a & 1]);
         a_pub[j] = a + 1;
-        progress = true;
       }
-      const int af = *reinterpret_cast<volatile int32_t*>(&pg.a_final);
+    }
+    for (int j = 0; j < kQGroups; j++) {
+      const int af = *reinterpret_cast<volatile int32_t*>(&sm.grp[j].a_final);
       if (af < 0 || a_pub[j] < af) all = false;
     }
     if (all) return;
-    if (progress) {
+    if (any) {
       idle = 0;
     } else if (++idle > kIdleLimit || ld_relaxed_u32(abort_word) != 0u) {
       return;  // the compute groups stop on their own bounded waits
     } else {
-      __nanosleep(64);
+      __nanosleep(256);  // leave the issue slots to the compute warps
     }
   }
 }
