@@ -69,77 +69,7 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float& lo, float& h
       : "=f"(lo), "=f"(hi) : "r"(h2));
 }
 
-// ------------------------------------------------------------- E2M1 codes
-
-// d = (a0 * b0, a1 * b1), one IEEE multiply per lane (packed on sm_100a)
-__device__ __forceinline__ void mul2(float a0, float a1, float b0, float b1, float& d0, float& d1) {
-  asm("{.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
-// Eight fp32 values -> one word of eight E2M1 codes; value 2j in the low
-// nibble of byte j (RNE, saturating at 6, sign kept).
-__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4,
-                                           float v5, float v6, float v7) {
-  uint32_t r;
-  asm("{.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};}"
-      : "=r"(r)
-      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
-  return r;
-}
-
-// Four pairs (lo_i, hi_i) -> one word whose byte i holds the pair's two
-// codes (lo_i in the low nibble).
-__device__ __forceinline__ uint32_t e2m1x2x4(float lo0, float hi0, float lo1, float hi1,
-                                             float lo2, float hi2, float lo3, float hi3) {
-  return e2m1x8(lo0, hi0, lo1, hi1, lo2, hi2, lo3, hi3);
-}
-
-// Row encode of eight bf16 (one 16-byte chunk = four words) with one
-// multiplier: the packed codes of the chunk.
-__device__ __forceinline__ uint32_t encode_chunk(const uint4& w, float enc) {
-  float y0, y1, y2, y3, y4, y5, y6, y7;
-  mul2(bf16lo(w.x), bf16hi(w.x), enc, enc, y0, y1);
-  mul2(bf16lo(w.y), bf16hi(w.y), enc, enc, y2, y3);
-  mul2(bf16lo(w.z), bf16hi(w.z), enc, enc, y4, y5);
-  mul2(bf16lo(w.w), bf16hi(w.w), enc, enc, y6, y7);
-  return e2m1x8(y0, y1, y2, y3, y4, y5, y6, y7);
-}
-
 // --------------------------------------------------------------- decoding
-
-// one word of eight E2M1 codes -> eight fp32 values (exact)
-__device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float (&v)[8]) {
-  uint32_t h0, h1, h2, h3;
-  asm("{.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3) : "r"(w));
-  const uint32_t h[4] = {h0, h1, h2, h3};
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-    float lo, hi;
-    asm("{.reg .f16 l, h;\n\t"
-        "mov.b32 {l, h}, %2;\n\t"
-        "cvt.f32.f16 %0, l;\n\t"
-        "cvt.f32.f16 %1, h;}"
-        : "=f"(lo), "=f"(hi) : "r"(h[i]));
-    v[2 * i] = lo;
-    v[2 * i + 1] = hi;
-  }
-}
 
 // one E4M3 byte -> fp32 (exact)
 __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
