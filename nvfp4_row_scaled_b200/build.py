@@ -13,6 +13,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libnvfp4rs.so")
+# the same library with -DNVFP4_TEST_HOOKS, loaded only by the timeout test
+TEST_LIB = os.path.join(HERE, "libnvfp4rs_test.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -28,19 +30,29 @@ def sources():
         os.path.join(INCLUDE, "nvfp4rs.h")]
 
 
-def build_library(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if it is missing or older than any source."""
-    if not force and os.path.exists(LIB):
-        if os.path.getmtime(LIB) >= max(os.path.getmtime(s) for s in sources()):
-            return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "nvfp4rs.cu")]
+def _build(lib: str, extra, force: bool, verbose: bool) -> str:
+    if not force and os.path.exists(lib):
+        if os.path.getmtime(lib) >= max(os.path.getmtime(s) for s in sources()):
+            return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [NVCC, *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "nvfp4rs.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_library(force: bool = False, verbose: bool = False) -> str:
+    """Compile the library if it is missing or older than any source."""
+    return _build(LIB, [], force, verbose)
+
+
+def build_test_library(force: bool = False) -> str:
+    """The library with its test hooks (see NVFP4_TEST_HOOKS in nvfp4rs.cu)."""
+    return _build(TEST_LIB, ["-DNVFP4_TEST_HOOKS"], force, False)
 
 
 if __name__ == "__main__":
     print(build_library(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build_test_library(force="--force" in sys.argv))

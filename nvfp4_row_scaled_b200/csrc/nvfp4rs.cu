@@ -308,6 +308,29 @@ nvfp4_status zero_quantize_state(void* workspace, int32_t E, float* row_acc, int
   return s;
 }
 
+#ifdef NVFP4_TEST_HOOKS
+// Test builds only (libnvfp4rs_test.so): the one-launch calls start their
+// item counter at this position instead of 0. The amax items before it are
+// then never claimed, so a cast item's bounded wait for its group runs out:
+// the test of the kernel's timeout path. The product library has no hook.
+uint8_t g_test_first_position = 0;
+
+// Sets the counter's first byte (the workspace header is zero just before).
+nvfp4_status test_hook_first_position(void* workspace, cudaStream_t stream) {
+  if (g_test_first_position == 0) return NVFP4_OK;
+  return cuda_status(cudaMemsetAsync(workspace, g_test_first_position, 1, stream));
+}
+#define NVFP4_TEST_HOOK(ws, stream)                                  \
+  do {                                                               \
+    const nvfp4_status hs = test_hook_first_position((ws), (stream)); \
+    if (hs != NVFP4_OK) return hs;                                   \
+  } while (0)
+#else
+#define NVFP4_TEST_HOOK(ws, stream) \
+  do {                              \
+  } while (0)
+#endif
+
 // ------------------------------------------------ scratch without allocation
 //
 // nvfp4_group_quantize_noalloc runs the one-launch kernel with its scratch in
@@ -547,6 +570,7 @@ nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
   // the rows accumulate straight into row_amax
   s = zero_quantize_state(workspace, num_groups, row_amax, sum_M, do_row, col_amax, K, do_col, stream);
   if (s != NVFP4_OK) return s;
+  NVFP4_TEST_HOOK(workspace, stream);
   return launch_quantize(routing, x_bf16, sum_M, K, num_groups, static_cast<uint32_t*>(workspace),
                          row_amax, row_amax, col_amax, out, do_col, stream);
 }
@@ -578,6 +602,7 @@ nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity
   s = zero_quantize_state(workspace, num_groups, row_acc, capacity_rows, do_row, col_amax, K, do_col,
                           stream);
   if (s != NVFP4_OK) return s;
+  NVFP4_TEST_HOOK(workspace, stream);
   return launch_quantize(routing, x_bf16, capacity_rows, K, num_groups,
                          static_cast<uint32_t*>(workspace), row_acc, row_amax, col_amax, out, do_col,
                          stream);
@@ -691,3 +716,7 @@ const char* nvfp4_status_string(nvfp4_status status) {
 }
 
 }  // extern "C"
+
+#ifdef NVFP4_TEST_HOOKS
+extern "C" NVFP4RS_API void nvfp4_test_set_first_position(uint8_t position) { g_test_first_position = position; }
+#endif
