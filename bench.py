@@ -211,6 +211,115 @@ def cpu_oracle_sample(w, target_s: float = 12.0, max_threads: int = 64):
                       f"one group per thread, {dt:.1f} s"}
 
 
+# ------------------------------------------------- the other configurations
+
+def other_configs(dev, steps: int):
+    """Amax + cast throughput on the other synthetic configurations, beside
+    the headline: the tiny and the 8-expert cases (inputs smaller than L2, so
+    L2 is flushed by writing 256 MB before each timed step), the graph-safe
+    case (the two graph-safe calls captured once in a CUDA graph and replayed
+    over its ten device routings), and the dense single-group case. Each
+    figure is the median of per-step CUDA-event times on the launching
+    stream."""
+    import torch
+
+    from nvfp4_row_scaled_b200 import abi, workloads
+
+    peak, _ = hbm_peak()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    n = max(steps, 10)
+
+    def median_ms(fn, flush_l2, before=None, reps=n):
+        evs = []
+        for i in range(reps):
+            if before is not None:
+                before(i)
+            if flush_l2:
+                flush.zero_()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+            evs.append((a0, a1))
+        torch.cuda.synchronize(dev)
+        return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+    def line(w, rows, ms, how):
+        b = algorithmic_bytes(rows, w.K, w.E)["step"]
+        return {"workload": w.name, "sum_M": rows, "K": w.K, "experts": w.E, "ms_per_step": round(ms, 4),
+                "value": round(rows * w.K / (ms * 1e-3) / 1e9, 3), "unit": "Gelem/s",
+                "hbm_gbs": round(b / (ms * 1e-3) / 1e9, 1),
+                "hbm_frac_of_peak": round(b / (ms * 1e-3) / 1e9 / peak, 4), "timing": how}
+
+    res = {}
+    for cid in (1, 2, 5):
+        w = workloads.make(cid)
+        x = w.x.to(dev)
+        R, K, E = w.sum_M, w.K, w.E
+        ra, ca = abi.alloc_amax(R, K, E, dev)
+        out = abi.alloc_outputs(R, K, E, dev)
+
+        def step():
+            abi.nvfp4_group_amax(x, w.m_splits, ra, ca)
+            abi.nvfp4_group_cast(x, w.m_splits, ra, ca, out)
+
+        for _ in range(3):
+            step()
+        small = 2 * R * K < 128 * 1024 * 1024
+        ms = median_ms(step, small)
+        res[f"config{cid}"] = line(w, R, ms, "host split; " + ("L2 flushed before each step" if small
+                                                               else "input larger than L2"))
+        del x, ra, ca, out
+
+    # graph-safe: routing only in device first_dims / tensor_offsets
+    w = workloads.config4()
+    x = w.x.to(dev)
+    cap, K, E = w.capacity_rows, w.K, w.E
+    fd = torch.zeros(E, dtype=torch.int64, device=dev)
+    offs = torch.zeros(E + 1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ra, ca = abi.alloc_amax(cap, K, E, dev)
+    out = abi.alloc_outputs(cap, K, E, dev)
+    routes = [abi.routing_tensors(r, K, dev) for r in w.routings]
+
+    def set_routing(i):
+        fd.copy_(routes[i % len(routes)][0])
+        offs.copy_(routes[i % len(routes)][1])
+
+    def gs_step():
+        abi.nvfp4_group_amax_graphsafe(x, fd, offs, ra, ca, status)
+        abi.nvfp4_group_cast_graphsafe(x, fd, offs, ra, ca, out, status)
+
+    set_routing(0)
+    gs_step()
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        gs_step()
+    for i in range(3):
+        set_routing(i)
+        graph.replay()
+    ms = median_ms(graph.replay, False, before=set_routing, reps=2 * len(routes))
+    if int(status.item()) != 0:
+        raise RuntimeError(f"graph-safe replay reported status {int(status.item())}")
+    res["config4"] = line(w, cap, ms, "CUDA-graph replay, routing rewritten on the device before each "
+                                      "replay (ten routings, twice); input larger than L2")
+
+    def hs_step():
+        abi.nvfp4_group_amax(x, w.routings[0], ra, ca)
+        abi.nvfp4_group_cast(x, w.routings[0], ra, ca, out)
+
+    for _ in range(3):
+        hs_step()
+    ms = median_ms(hs_step, False)
+    res["config4_host_split"] = line(w, cap, ms, "the same input and its first routing through the host-split "
+                                                 "calls; input larger than L2")
+    del graph, x, ra, ca, out, flush
+    return res
+
+
 # --------------------------------------------------------------- the bench
 
 def main():
@@ -221,6 +330,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tokens", type=int, default=8192, help="scales the workload (tests only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the throughput of configurations other than the headline one")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -445,6 +556,9 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(w)
+    others = None
+    if world == 1 and not args.no_other_configs:
+        others = other_configs(dev, args.steps)
 
     line = {
         "metric": METRIC,
@@ -524,6 +638,7 @@ def main():
                       "hbm_gbs": round(deq_mx_bytes / (deq_mx_ms * 1e-3) / 1e9, 1),
                       "hbm_frac_of_peak": round(deq_mx_bytes / (deq_mx_ms * 1e-3) / 1e9 / peak, 4)},
         },
+        "other_configs": others,
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
