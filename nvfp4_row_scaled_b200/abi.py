@@ -23,7 +23,9 @@ from typing import Dict, Optional, Sequence
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnvfp4rs.so")
+# NVFP4RS_LIBRARY names another build of the same library to load instead
+# (the bounds-checked debug build, libnvfp4rs_debug.so, for instance)
+LIB_PATH = os.environ.get("NVFP4RS_LIBRARY") or os.path.join(HERE, "libnvfp4rs.so")
 
 NVFP4_OK = 0
 NVFP4_ERR_INVALID_ARG = 1

@@ -15,6 +15,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libnvfp4rs.so")
 # the same library with -DNVFP4_TEST_HOOKS, loaded only by the timeout test
 TEST_LIB = os.path.join(HERE, "libnvfp4rs_test.so")
+# the bounds-checked debug build (-DNVFP4_CHECK_BOUNDS, see csrc/bounds.cuh)
+DEBUG_LIB = os.path.join(HERE, "libnvfp4rs_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -53,6 +55,13 @@ def build_test_library(force: bool = False) -> str:
     return _build(TEST_LIB, ["-DNVFP4_TEST_HOOKS"], force, False)
 
 
+def build_debug_library(force: bool = False) -> str:
+    """The bounds-checked debug build: every global access of the kernels is
+    checked against the ranges registered for its launch."""
+    return _build(DEBUG_LIB, ["-DNVFP4_CHECK_BOUNDS"], force, False)
+
+
 if __name__ == "__main__":
     print(build_library(force="--force" in sys.argv, verbose="-v" in sys.argv))
     print(build_test_library(force="--force" in sys.argv))
+    print(build_debug_library(force="--force" in sys.argv))

@@ -15,6 +15,7 @@
 // load and one scale byte; no division.
 #pragma once
 
+#include "bounds.cuh"
 #include "codec.cuh"
 
 namespace nvfp4rs {
@@ -55,12 +56,12 @@ dequant_kernel(const uint16_t* __restrict__ data, const uint8_t* __restrict__ sc
        r += warps) {
     const uint16_t* d = data + r * cols4;
     const uint8_t* sc = scale + r * spr;
-    const float sd = kMx ? 1.0f : s2[r];
+    const float sd = kMx ? 1.0f : gload(&s2[r]);
     float4* o = out + r * cols4;
 #pragma unroll 4
     for (int64_t q = lane; q < cols4; q += 32) {
-      const uint16_t c = d[q];
-      const uint32_t sb = sc[kMx ? (q >> 3) : (q >> 2)];
+      const uint16_t c = gload(&d[q]);
+      const uint32_t sb = gload(&sc[kMx ? (q >> 3) : (q >> 2)]);
       float v[4];
       e2m1x4_to_f32(c, v);
       float4 y;
@@ -73,7 +74,7 @@ dequant_kernel(const uint16_t* __restrict__ data, const uint8_t* __restrict__ sc
         y = make_float4(__fmul_rn(__fmul_rn(v[0], sv), sd), __fmul_rn(__fmul_rn(v[1], sv), sd),
                         __fmul_rn(__fmul_rn(v[2], sv), sd), __fmul_rn(__fmul_rn(v[3], sv), sd));
       }
-      __stcs(o + q, y);
+      if (NVFP4_STORE_OK(o + q, 16)) __stcs(o + q, y);
     }
   }
 }

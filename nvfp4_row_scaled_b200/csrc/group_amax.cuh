@@ -47,6 +47,7 @@ constexpr int kAmaxThreads = 128;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
+  if (!NVFP4_LOAD_OK(p, 16)) return make_uint4(0u, 0u, 0u, 0u);
   asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
       : "l"(p));
@@ -54,6 +55,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 }
 
 __device__ __forceinline__ void red_max_u32(float* addr, uint32_t v) {
+  if (!NVFP4_STORE_OK(addr, 4)) return;
   asm volatile("red.global.max.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
 }
 
@@ -190,7 +192,7 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   if (active && rank == 0 && row_amax != nullptr && t < valid) {
     uint32_t m = rmax[t];
     for (int q = 1; q < cn; q++) m = max(m, *cluster.map_shared_rank(&rmax[t], q));
-    row_amax[r0 + t] = __uint_as_float(m);
+    gstore(&row_amax[r0 + t], __uint_as_float(m));
   }
   cluster.sync();
 }

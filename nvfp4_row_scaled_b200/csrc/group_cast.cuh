@@ -138,10 +138,12 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 __device__ __forceinline__ void st_global_u2_hint(void* p, uint2 v, uint64_t policy) {
+  if (!NVFP4_STORE_OK(p, 8)) return;
   asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y),
                "l"(policy) : "memory");
 }
 __device__ __forceinline__ void st_global_u4_hint(void* p, uint4 v, uint64_t policy) {
+  if (!NVFP4_STORE_OK(p, 16)) return;
   asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy) : "memory");
 }
@@ -172,6 +174,7 @@ __device__ __forceinline__ void issue_tile_at(CastSmem& sm, const CUtensorMap* m
 // Untiled bulk copy global -> shared (16-byte aligned, multiple of 16 bytes),
 // completion counted on `bar`. No multicast.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  src = NVFP4_BULK_SRC(src, bytes);
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_addr(dst)),
@@ -197,7 +200,7 @@ __device__ __forceinline__ void load_patch(const uint8_t* tile, int cc, int rl, 
 }
 
 __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
-  *reinterpret_cast<uint32_t*>(p) = v;
+  gstore(reinterpret_cast<uint32_t*>(p), v);
 }
 
 // The codes of a lane's 16 x 8 patch, once the multipliers are known: renc[i]
@@ -485,7 +488,7 @@ __device__ __forceinline__ void store_staged_single(const CastStage& st, const C
       const int sw = (col >> 3) & 7;
       st_global_u2_hint(gd + static_cast<size_t>(c0 + col) * half_m + 8 * b,
                         *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * (b ^ sw)]), keep);
-      gs[static_cast<size_t>(c0 + col) * m16 + b] = st.col_scale[b * kCols + col];
+      gstore(&gs[static_cast<size_t>(c0 + col) * m16 + b], st.col_scale[b * kCols + col]);
     }
   }
   if (do_row) {
@@ -525,8 +528,8 @@ __device__ __noinline__ void store_staged_general(const CastStage& st, const Cas
       st_global_u2_hint(out.col_data + (static_cast<size_t>(K) * o >> 1) + static_cast<size_t>(c0 + col) * (m >> 1) +
                             ((r - o) >> 1),
                         d, keep);
-      out.col_scale[(static_cast<size_t>(K) * o >> 4) + static_cast<size_t>(c0 + col) * (m >> 4) + ((r - o) >> 4)] =
-          st.col_scale[b * kCols + col];
+      gstore(&out.col_scale[(static_cast<size_t>(K) * o >> 4) + static_cast<size_t>(c0 + col) * (m >> 4) + ((r - o) >> 4)],
+             st.col_scale[b * kCols + col]);
     }
   }
   if (do_row && t < valid) {
@@ -574,7 +577,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
     const int64_t n = static_cast<int64_t>(rs.E) * K;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kCastThreads + t; i < n;
          i += static_cast<int64_t>(gridDim.x) * kCastThreads)
-      out.col_s2[i] = s_dec_of(col_amax[i]);
+      gstore(&out.col_s2[i], s_dec_of(gload(&col_amax[i])));
   }
   sm.e4m3[t] = e4m3_entry(t);
 
@@ -622,17 +625,17 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
       m_g = rs.off[g + 1] - o_g;
       if (do_row) {
         const bool in = t < valid;
-        const float a = in ? row_amax[r0 + t] : 0.0f;
+        const float a = in ? gload(&row_amax[r0 + t]) : 0.0f;
         sm.row_senc[t] = s_enc_of(a);
         row_slow = in && !fast_path_amax(a);
-        if (ct == 0 && in) out.row_s2[r0 + t] = s_dec_of(a);
+        if (ct == 0 && in) gstore(&out.row_s2[r0 + t], s_dec_of(a));
       }
     }
     slow |= row_slow;
     const bool mixed = o_g + m_g < r0 + valid;  // the tile crosses a group boundary
     if (do_col) {
       if (!mixed) {
-        const float a = col_amax[static_cast<size_t>(g) * K + c0 + t];
+        const float a = gload(&col_amax[static_cast<size_t>(g) * K + c0 + t]);
         sm.col_senc[0][t] = s_enc_of(a);
         slow |= !fast_path_amax(a);
       } else {  // one column table per 16-row block, from the block's group
@@ -641,7 +644,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
         for (int b = 0; kBlockRows * b < valid; b++) {
           while (rs.off[gb + 1] <= r0 + kBlockRows * b) gb++;  // groups only move forward
           if (gb != gprev) {  // a new group (a tile holds few): its column scale
-            const float a = col_amax[static_cast<size_t>(gb) * K + c0 + t];
+            const float a = gload(&col_amax[static_cast<size_t>(gb) * K + c0 + t]);
             e = s_enc_of(a);
             slow |= !fast_path_amax(a);
             gprev = gb;

@@ -163,7 +163,7 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
 #pragma unroll 4
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kPThreads + t; i < n;
          i += static_cast<int64_t>(gridDim.x) * kPThreads)
-      out.col_s2[i] = s_dec_of(col_amax[i]);
+      gstore(&out.col_s2[i], s_dec_of(gload(&col_amax[i])));
   }
 
   const int lane = gt & 31, w = gt >> 5;
@@ -191,7 +191,7 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
         const float a = pg.row_senc[slot][gt];
         pg.row_senc[slot][gt] = s_enc_of(a);
         slow |= !fast_path_amax(a);
-        if (ct == 0) out.row_s2[r0 + gt] = s_dec_of(a);
+        if (ct == 0) gstore(&out.row_s2[r0 + gt], s_dec_of(a));
       }
       if (do_col) {
         const float a = pg.col_senc[slot][gt];

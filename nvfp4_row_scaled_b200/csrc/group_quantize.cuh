@@ -84,17 +84,27 @@ constexpr int64_t quant_ws_header_words(int64_t E) { return (kWsDone + E + 63) /
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
+  if (!NVFP4_LOAD_OK(p, 4)) return 0u;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
   uint32_t v;
+  if (!NVFP4_LOAD_OK(p, 4)) return 0u;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
-__device__ __forceinline__ void raise_abort(uint32_t* abort_word) { atomicExch(abort_word, 1u); }
+__device__ __forceinline__ void raise_abort(uint32_t* abort_word) {
+  if (NVFP4_STORE_OK(abort_word, 4)) atomicExch(abort_word, 1u);
+}
+
+// Claim the next sequence position (past the end of any sequence when the
+// counter is out of bounds in the checked build).
+__device__ __forceinline__ uint32_t claim(uint32_t* counter) {
+  return NVFP4_STORE_OK(counter, 4) ? atomicAdd(counter, 1u) : 0xFFFFFFFFu;
+}
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
@@ -231,8 +241,8 @@ __device__ __forceinline__ void quantize_producer(QuantSmem& sm, int j, const Ro
   const uint32_t n = static_cast<uint32_t>(rs.total >> 7) * static_cast<uint32_t>(n_ct);
   const uint32_t amax_bytes = (do_row ? 512u : 0u) + (do_col ? 512u : 0u);
   ItemCursor cur;
-  uint32_t q0 = atomicAdd(counter, 1u);  // the next position to issue
-  uint32_t q1 = atomicAdd(counter, 1u);  // the one after it
+  uint32_t q0 = claim(counter);  // the next position to issue
+  uint32_t q1 = claim(counter);  // the one after it
   bool fail = false;
   int i = 0;  // items issued
   for (;; i++) {
@@ -252,7 +262,7 @@ __device__ __forceinline__ void quantize_producer(QuantSmem& sm, int j, const Ro
       break;
     }
     q0 = q1;
-    q1 = atomicAdd(counter, 1u);
+    q1 = claim(counter);
     const bool is_b = (item & kBItem) != 0;
     const int tl = item_tile(item);
     const int rt = tl / n_ct, ct = tl - rt * n_ct;
@@ -318,7 +328,8 @@ __device__ __forceinline__ void quantize_publisher(QuantSmem& sm, uint32_t* ws) 
         QuantGroup& pg = sm.grp[j];
         const int a = a_pub[j];
         const int g = reinterpret_cast<volatile int32_t*>(pg.pub_grp)[a & 3];
-        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(&done[g]) : "memory");
+        if (NVFP4_STORE_OK(&done[g], 4))
+          asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(&done[g]) : "memory");
         mbar_arrive(&pg.aack[a & 1]);
         a_pub[j] = a + 1;
       }
@@ -372,7 +383,7 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
   if (do_col) {  // empty groups own no tile: their col_s2 is S_dec(0) (col_amax stays 0)
     for (int g = blockIdx.x; g < E; g += gridDim.x)
       if (off[g + 1] == off[g])
-        for (int c = t; c < K; c += kQThreads) out.col_s2[static_cast<size_t>(g) * K + c] = s_dec_of(0.0f);
+        for (int c = t; c < K; c += kQThreads) gstore(&out.col_s2[static_cast<size_t>(g) * K + c], s_dec_of(0.0f));
   }
   if (t < 128) sm.e4m3[t] = e4m3_entry(t);
   if (t == 0) {
@@ -441,15 +452,15 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
         pg.row_senc[s][gt] = s_enc_of(a);
         slow |= !fast_path_amax(a);
         if (ct == 0) {
-          if (row_amax != row_acc) row_amax[r0 + gt] = a;
-          out.row_s2[r0 + gt] = s_dec_of(a);
+          if (row_amax != row_acc) gstore(&row_amax[r0 + gt], a);
+          gstore(&out.row_s2[r0 + gt], s_dec_of(a));
         }
       }
       if (do_col) {
         const float a = pg.col_amax[s][gt];
         pg.col_senc[s][gt] = s_enc_of(a);
         slow |= !fast_path_amax(a);
-        if (r0 == rs.off[g]) out.col_s2[static_cast<size_t>(g) * K + c0 + gt] = s_dec_of(a);
+        if (r0 == rs.off[g]) gstore(&out.col_s2[static_cast<size_t>(g) * K + c0 + gt], s_dec_of(a));
       }
     }
     if (item == kAbortItem) pg.fail = 1;

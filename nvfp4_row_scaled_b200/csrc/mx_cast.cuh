@@ -174,14 +174,16 @@ mx_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ 
       const uint32_t w = static_cast<uint32_t>(st.col_scale[t]) | (static_cast<uint32_t>(st.col_scale[kCols + t]) << 8) |
                          (static_cast<uint32_t>(st.col_scale[2 * kCols + t]) << 16) |
                          (static_cast<uint32_t>(st.col_scale[3 * kCols + t]) << 24);
-      *reinterpret_cast<uint32_t*>(out.col_scale + (static_cast<size_t>(K) * o_g >> 5) +
-                                   static_cast<size_t>(c0 + t) * (static_cast<size_t>(m_g) >> 5) + ((r0 - o_g) >> 5)) = w;
+      gstore(reinterpret_cast<uint32_t*>(out.col_scale + (static_cast<size_t>(K) * o_g >> 5) +
+                                         static_cast<size_t>(c0 + t) * (static_cast<size_t>(m_g) >> 5) +
+                                         ((r0 - o_g) >> 5)),
+             w);
     }
     if (do_row) {
       const uint32_t w = static_cast<uint32_t>(st.row_scale[t]) | (static_cast<uint32_t>(st.row_scale[kRows + t]) << 8) |
                          (static_cast<uint32_t>(st.row_scale[2 * kRows + t]) << 16) |
                          (static_cast<uint32_t>(st.row_scale[3 * kRows + t]) << 24);
-      *reinterpret_cast<uint32_t*>(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 5) + (c0 >> 5)) = w;
+      gstore(reinterpret_cast<uint32_t*>(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 5) + (c0 >> 5)), w);
     }
   }
   if (failed && t == 0) {

@@ -38,6 +38,52 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
+#ifdef NVFP4_CHECK_BOUNDS
+// The checked debug build: the byte ranges a launch may touch, registered on
+// its stream just before it (see bounds.cuh). The first range must be an
+// input of at least 512 bytes (x) wherever the kernel makes bulk copies.
+struct SpanList {
+  Spans s{};
+  bool overflow = false;
+  SpanList& add(const void* p, size_t bytes, bool store) {
+    if (p != nullptr && bytes > 0 && s.n == kMaxSpans) overflow = true;
+    if (p != nullptr && bytes > 0 && s.n < kMaxSpans) {
+      s.lo[s.n] = reinterpret_cast<uint64_t>(p);
+      s.hi[s.n] = s.lo[s.n] + bytes;
+      s.store[s.n] = store ? 1u : 0u;
+      s.n++;
+    }
+    return *this;
+  }
+  SpanList& routing(const HostRouting&) { return *this; }
+  SpanList& routing(const DeviceRouting& r) {
+    if (r.uniform_rows >= 0) return add(r.status, 4, true);
+    return add(r.first_dims, static_cast<size_t>(r.E) * 8, false)
+        .add(r.tensor_offsets, static_cast<size_t>(r.E + 1) * 8, false)
+        .add(r.status, 4, true);
+  }
+  SpanList& outputs(const CastOut& o, int64_t rows, int64_t K, int32_t E) {
+    const size_t n = static_cast<size_t>(rows) * static_cast<size_t>(K);
+    return add(o.row_data, n / 2, true).add(o.row_scale, n / 16, true).add(o.row_s2, 4 * static_cast<size_t>(rows), true)
+        .add(o.col_data, n / 2, true).add(o.col_scale, n / 16, true).add(o.col_s2, 4 * static_cast<size_t>(E) * K, true);
+  }
+  nvfp4_status set(cudaStream_t stream) const {
+    if (overflow) return NVFP4_ERR_UNSUPPORTED;  // more ranges than the table holds
+    set_spans_kernel<<<1, 1, 0, stream>>>(s);
+    return cuda_status(cudaGetLastError());
+  }
+};
+#define NVFP4_SPANS(expr)                           \
+  do {                                              \
+    const nvfp4_status span_status = (expr);        \
+    if (span_status != NVFP4_OK) return span_status; \
+  } while (0)
+#else
+#define NVFP4_SPANS(expr) \
+  do {                    \
+  } while (0)
+#endif
+
 // CTAs per cluster along K for the amax kernel: the largest d <= 8 that
 // divides the number of 128-column chunks.
 int amax_cluster(int64_t K) {
@@ -162,9 +208,16 @@ bool x_tensor_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K) {
 }
 
 template <class Routing>
-nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t tiles, int64_t K, int32_t E,
+nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
                          float* row_amax, float* col_amax, cudaStream_t stream) {
+  const int64_t tiles = (rows + kRows - 1) / kRows;
   if (tiles == 0 || K == 0) return NVFP4_OK;
+  NVFP4_SPANS(SpanList{}
+                  .add(x, static_cast<size_t>(rows) * K * 2, false)
+                  .routing(routing)
+                  .add(row_amax, 4 * static_cast<size_t>(rows), true)
+                  .add(col_amax, 4 * static_cast<size_t>(E) * K, true)
+                  .set(stream));
   const int cn = amax_cluster(K);
   const size_t smem = static_cast<size_t>(K / cn) * sizeof(uint32_t) + sizeof(int32_t) * (E + 1);
   auto kernel = group_amax_kernel<Routing>;
@@ -226,6 +279,13 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
   if (grid < 1) grid = 1;
   CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2,
             out->scale_layout == NVFP4_SCALE_TILED_128X4};
+  NVFP4_SPANS(SpanList{}
+                  .add(x, static_cast<size_t>(rows) * K * 2, false)
+                  .routing(routing)
+                  .add(row_amax, 4 * static_cast<size_t>(rows), false)
+                  .add(col_amax, 4 * static_cast<size_t>(E) * K, false)
+                  .outputs(o, rows, K, E)
+                  .set(stream));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(threads);
@@ -270,6 +330,15 @@ nvfp4_status launch_quantize(const Routing& routing, const void* x, int64_t rows
   const int32_t lag = static_cast<int32_t>(kQuantLagRounds * kQGroups * grid);
   CastOut o{out->row_data, out->row_scale, out->row_s2, out->col_data, out->col_scale, out->col_s2,
             out->scale_layout == NVFP4_SCALE_TILED_128X4};
+  NVFP4_SPANS(SpanList{}
+                  .add(x, static_cast<size_t>(rows) * K * 2, false)
+                  .routing(routing)
+                  .add(ws, 4 * static_cast<size_t>(quant_ws_header_words(E)), true)
+                  .add(row_acc, 4 * static_cast<size_t>(rows), true)
+                  .add(row_amax, 4 * static_cast<size_t>(rows), true)
+                  .add(col_amax, 4 * static_cast<size_t>(E) * K, true)
+                  .outputs(o, rows, K, E)
+                  .set(stream));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kQThreads);
@@ -399,6 +468,19 @@ nvfp4_status launch_mx_cast(const Routing& routing, const void* x, int64_t rows,
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
   if (tiles < grid) grid = tiles;
   const MxOut o{out->row_data, out->row_scale, out->col_data, out->col_scale};
+#ifdef NVFP4_CHECK_BOUNDS
+  {
+    const size_t n = static_cast<size_t>(rows) * K;
+    NVFP4_SPANS(SpanList{}
+                    .add(x, n * 2, false)
+                    .routing(routing)
+                    .add(o.row_data, n / 2, true)
+                    .add(o.row_scale, n / 32, true)
+                    .add(o.col_data, n / 2, true)
+                    .add(o.col_scale, n / 32, true)
+                    .set(stream));
+  }
+#endif
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kCastThreads);
@@ -415,6 +497,17 @@ nvfp4_status launch_dequant(const uint8_t* data, const uint8_t* scale, const flo
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t rows_per_cta = kDequantThreads / 32;
   int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
+#ifdef NVFP4_CHECK_BOUNDS
+  {
+    const size_t n = static_cast<size_t>(rows) * static_cast<size_t>(cols);
+    NVFP4_SPANS(SpanList{}
+                    .add(data, n / 2, false)
+                    .add(scale, kMx ? n / 32 : n / 16, false)
+                    .add(s2, kMx ? 0 : 4 * static_cast<size_t>(rows), false)
+                    .add(out_f32, n * 4, true)
+                    .set(stream));
+  }
+#endif
   if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -443,8 +536,7 @@ nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
                                     stream));
     if (s != NVFP4_OK) return s;
   }
-  return launch_amax(routing, x_bf16, (sum_M + kRows - 1) / kRows, K, num_groups, row_amax, col_amax,
-                     stream);
+  return launch_amax(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, stream);
 }
 
 nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
@@ -491,8 +583,7 @@ nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_row
     if (s != NVFP4_OK) return s;
   }
   if (K == 0) return NVFP4_OK;
-  return launch_amax(routing, x_bf16, (capacity_rows + kRows - 1) / kRows, K, num_groups, row_amax,
-                     col_amax, stream);
+  return launch_amax(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, stream);
 }
 
 nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
@@ -652,6 +743,17 @@ nvfp4_status nvfp4_row_post_scale(const float* gemm_out, int64_t rows, int64_t c
   const int64_t cap = static_cast<int64_t>(sms) * 2;  // persistent: two CTAs per SM are resident
   if (grid > cap) grid = cap;
   const bool b16 = out_dtype == NVFP4_OUT_BF16, has_bias = bias != nullptr;
+#ifdef NVFP4_CHECK_BOUNDS
+  {
+    const size_t n = static_cast<size_t>(rows) * static_cast<size_t>(cols);
+    NVFP4_SPANS(SpanList{}
+                    .add(gemm_out, n * 4, false)
+                    .add(row_amax, 4 * static_cast<size_t>(rows), false)
+                    .add(bias, 4 * static_cast<size_t>(cols), false)
+                    .add(out, n * (b16 ? 2 : 4), true)
+                    .set(stream));
+  }
+#endif
   auto kernel = b16 ? (has_bias ? row_post_scale_kernel<true, true> : row_post_scale_kernel<true, false>)
                     : (has_bias ? row_post_scale_kernel<false, true> : row_post_scale_kernel<false, false>);
   cudaLaunchConfig_t cfg = {};
@@ -719,4 +821,18 @@ const char* nvfp4_status_string(nvfp4_status status) {
 
 #ifdef NVFP4_TEST_HOOKS
 extern "C" NVFP4RS_API void nvfp4_test_set_first_position(uint8_t position) { g_test_first_position = position; }
+#endif
+
+#ifdef NVFP4_CHECK_BOUNDS
+// The checked debug build only: accesses counted outside their launch's
+// registered ranges since load (or the last reset).
+extern "C" NVFP4RS_API unsigned long long nvfp4_debug_bounds_faults(void) {
+  unsigned long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, nvfp4rs::g_bounds_faults, sizeof(v)) != cudaSuccess) return ~0ull;
+  return v;
+}
+extern "C" NVFP4RS_API int nvfp4_debug_bounds_reset(void) {
+  const unsigned long long z = 0;
+  return cudaMemcpyToSymbol(nvfp4rs::g_bounds_faults, &z, sizeof(z)) == cudaSuccess ? 0 : 1;
+}
 #endif

@@ -19,12 +19,15 @@
 
 #include <cstdint>
 
+#include "bounds.cuh"
+
 namespace nvfp4rs {
 
 constexpr int kPostThreads = 256;
 
 __device__ __forceinline__ float4 ld_stream_f4(const float4* p) {
   float4 v;
+  if (!NVFP4_LOAD_OK(p, 16)) return make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   asm("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
       : "l"(p));
@@ -54,9 +57,9 @@ row_post_scale_kernel(const float4* in, int64_t rows, int64_t cols4, const float
     const int64_t r0 = rb * kPostUnitRows;
     const int64_t c = cb * 32 + lane;
     const int nr = rows - r0 < kPostUnitRows ? static_cast<int>(rows - r0) : kPostUnitRows;
-    const float a_lane = lane < nr ? amax[r0 + lane] : 0.0f;
+    const float a_lane = lane < nr ? gload(&amax[r0 + lane]) : 0.0f;
     float4 b = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (kBias && c < cols4) b = bias[c];
+    if (kBias && c < cols4) b = gload(&bias[c]);
     float4 x[kPostUnitRows];
 #pragma unroll
     for (int i = 0; i < kPostUnitRows; i++)
@@ -71,8 +74,8 @@ row_post_scale_kernel(const float4* in, int64_t rows, int64_t cols4, const float
           y = make_float4(__fadd_rn(y.x, b.x), __fadd_rn(y.y, b.y), __fadd_rn(y.z, b.z), __fadd_rn(y.w, b.w));
         const int64_t o = (r0 + i) * cols4 + c;
         if (kBf16)
-          reinterpret_cast<uint2*>(out)[o] = make_uint2(bf16x2_rn(y.x, y.y), bf16x2_rn(y.z, y.w));
-        else
+          gstore(reinterpret_cast<uint2*>(out) + o, make_uint2(bf16x2_rn(y.x, y.y), bf16x2_rn(y.z, y.w)));
+        else if (NVFP4_STORE_OK(reinterpret_cast<float4*>(out) + o, 16))
           __stcs(reinterpret_cast<float4*>(out) + o, y);
       }
     }

@@ -19,6 +19,7 @@
 #include <cstdint>
 
 #include "nvfp4rs.h"
+#include "bounds.cuh"
 
 namespace nvfp4rs {
 
@@ -89,15 +90,15 @@ struct DeviceRouting {
     }
     int bad_routing = 0, bad_align = 0, not_128 = 0;
     for (int i = threadIdx.x; i <= E; i += blockDim.x) {
-      const int64_t o = tensor_offsets[i];
+      const int64_t o = gload(&tensor_offsets[i]);
       if ((i == 0 && o != 0) || o < 0 || o % K != 0 || o / K > capacity_rows) {
         bad_routing = 1;
       } else {
         off_smem[i] = static_cast<int32_t>(o / K);
       }
       if (i < E) {
-        const int64_t fd = first_dims[i];
-        const int64_t next = tensor_offsets[i + 1];
+        const int64_t fd = gload(&first_dims[i]);
+        const int64_t next = gload(&tensor_offsets[i + 1]);
         if (fd < 0 || fd > capacity_rows || next - o != fd * K) bad_routing = 1;
         if (fd % align != 0) bad_align = 1;
         if (fd % kRows != 0) not_128 = 1;
@@ -113,11 +114,13 @@ struct DeviceRouting {
       s.E = E;
       s.ok = code == 0 && !skip;
       s.total = code == 0 ? off_smem[E] : 0;
-      if (code != 0) *status = code;
+      if (code != 0) gstore(status, static_cast<int32_t>(code));
     }
     __syncthreads();
   }
-  __device__ __forceinline__ void report(int code) const { atomicCAS(status, 0, code); }
+  __device__ __forceinline__ void report(int code) const {
+    if (NVFP4_STORE_OK(status, 4)) atomicCAS(status, 0, code);
+  }
 };
 
 // Group holding row r (r < total): the last g with off[g] <= r. Empty groups
