@@ -216,10 +216,11 @@ NVFP4RS_API size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, i
  * exactly what nvfp4_group_amax followed by nvfp4_group_cast computes
  * (TransformerEngine #3649, Description: the amax step's row and column amax
  * vectors are the cast step's scale sources) -- row_amax, col_amax and every
- * output of `out` byte-identical to that pair -- but reads each tile of x
- * from DRAM once: a persistent kernel runs the amax of a tile, and the cast
- * of the same tile a little later while it is still in L2, once all amax
- * work of its group has finished.
+ * output of `out` byte-identical to that pair -- but meant to read each tile
+ * of x from DRAM once: a persistent kernel runs the amax of a tile, and the
+ * cast of the same tile a little later while it is still in L2, once all
+ * amax work of its group has finished. A group too large for L2 between its
+ * two passes is read back in part.
  *   x_bf16, sum_M, K, m_splits_host, num_groups, out
  *                   as for nvfp4_group_cast
  *   row_amax        device fp32 [sum_M], written (needed when the row
