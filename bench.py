@@ -14,7 +14,7 @@ local experts; no collective on the data path) and rank 0 prints one JSON line.
 
 Metric: input Gelem/s (sum_M*K elements per step). Reported beside it: HBM
 GB/s of the method's algorithmic bytes and the roofline of the dominant
-kernel against the measured HBM copy bandwidth of this machine's B200s.
+kernel against the measured HBM copy bandwidth of the B200 (MEASURED_PEAKS.json).
 """
 from __future__ import annotations
 
