@@ -8,9 +8,11 @@ tokens x top-8 = 65536 routed rows, Zipf(1.1) expert popularity, ~10% empty
 experts, every group zero-padded to a multiple of 128 rows (synthetic, seeded).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-For N > 1 launch one process per GPU with torch.distributed.run; every rank
-casts its own copy of the workload (expert parallelism: each GPU casts its
-local experts; no collective on the data path) and rank 0 prints one JSON line.
+For N > 1 there is one process per GPU: either launch them with
+torch.distributed.run (WORLD_SIZE must equal N), or run `bench.py --gpus N`
+as one process and it starts the N ranks itself. Every rank casts its own
+copy of the workload (expert parallelism: each GPU casts its local experts;
+no collective on the data path) and rank 0 prints one JSON line.
 
 Metric: input Gelem/s (sum_M*K elements per step). Reported beside it: HBM
 GB/s of the method's algorithmic bytes and the roofline of the dominant
@@ -107,6 +109,22 @@ def job_throughput(elements_per_rank: int, world: int, ms_per_step: float) -> fl
     return world * elements_per_rank / (ms_per_step * 1e-3) / 1e9
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(n: int, argv) -> int:
+    """`bench.py --gpus N` started as one process: start N ranks of this
+    script, one per GPU, through torch.distributed.run on 127.0.0.1, and
+    return their exit status. Rank 0 prints the JSON line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd).returncode
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -168,10 +186,19 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle
 
+def host_cores() -> int:
+    """Cores this process may run on (the affinity mask, else the count)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def cpu_oracle_sample(w, target_s: float = 12.0, max_threads: int = 64):
     """Time the oracle (amax + cast, both directions) on a bounded sample of
     the workload: whole groups, taken in order until the sample has about
-    target_s of CPU work, run one group per thread across the host cores."""
+    target_s of CPU work, run one group per thread across the host cores
+    (max_threads=1: one thread, groups one after another)."""
     import numpy as np  # noqa: F401
 
     import oracle
@@ -180,7 +207,7 @@ def cpu_oracle_sample(w, target_s: float = 12.0, max_threads: int = 64):
     xb = workloads.bits(w.x)
     offs = workloads.row_offsets(w.m_splits)
     groups = [(offs[g], m) for g, m in enumerate(w.m_splits) if m > 0]
-    cores = min(os.cpu_count() or 1, max_threads)
+    cores = min(host_cores(), max_threads)
 
     def one(o_m):
         o, m = o_m
@@ -208,7 +235,18 @@ def cpu_oracle_sample(w, target_s: float = 12.0, max_threads: int = 64):
     return {"value": done / dt / 1e9, "unit": "Gelem/s", "cores": cores, "kind": "oracle",
             "sample": f"{len(sample)} whole groups ({sum(m for _, m in sample)} rows x {w.K}, "
                       f"{done / 1e6:.1f} M elements) of the workload, amax + cast both directions, "
-                      f"one group per thread, {dt:.1f} s"}
+                      f"one group per thread on {cores} thread(s), {dt:.1f} s"}
+
+
+def cpu_baseline(w):
+    """The oracle on the host cores (all of them, one group per thread) and on
+    one thread, each on a bounded sample of the workload."""
+    multi = cpu_oracle_sample(w)
+    single = cpu_oracle_sample(w, target_s=6.0, max_threads=1)
+    multi["nproc"] = host_cores()
+    multi["single_thread"] = {"value": single["value"], "unit": single["unit"], "cores": 1,
+                              "sample": single["sample"]}
+    return multi
 
 
 # ------------------------------------------------- the other configurations
@@ -324,7 +362,8 @@ def other_configs(dev, steps: int):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks, one per GPU; started through torch.distributed.run when WORLD_SIZE is unset")
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -336,9 +375,13 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(args.gpus, sys.argv[1:])
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
 
     if args.impl == "reference":
         return reference_arm(args, rank, world)
@@ -492,7 +535,7 @@ def main():
     # all its outputs back. Two device buffer sets on three streams let step
     # i+1's upload run while step i's outputs come back (PCIe is full duplex);
     # a buffer set is reused only after its previous step's download ended.
-    e2e_steps = max(3, min(args.steps, 5))
+    e2e_steps = args.steps
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
     xs = [x, torch.empty_like(x)]
     outs = [out, abi.alloc_outputs(M, K, E, dev)]
@@ -555,7 +598,7 @@ def main():
     traffic = traffic_record(dom_kernel, workload_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(w)
+        cpu = cpu_baseline(w)
     others = None
     if world == 1 and not args.no_other_configs:
         others = other_configs(dev, args.steps)
@@ -595,6 +638,9 @@ def main():
             "frac": round(achieved / peak, 4),
             "traffic": traffic,
             "algorithmic_bytes_per_launch": b[dominant],
+            "note": "per-kernel time: the cast's outputs carry an L2 evict-last hint, so part of its "
+                    "DRAM writes lands after it ends (inside the next step's amax launch); the step "
+                    "figure (hbm_frac_of_peak) includes that cost",
         },
         "cpu_baseline": cpu,
         "e2e": {
@@ -678,4 +724,4 @@ def reference_arm(args, rank: int, world: int):
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main() or 0)

@@ -275,7 +275,15 @@ NVFP4RS_API nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int6
  *     NVFP4_MAX_GROUPS groups; larger num_groups is NVFP4_ERR_UNSUPPORTED.
  *   - Setup: the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture. The cached address belongs
+ *     to the device's current context: after cudaDeviceReset on a device,
+ *     this call must not be used on that device again in the same process.
+ *   - Give-up: if a bounded wait inside the kernel gives up (not expected;
+ *     it needs a stalled SM elsewhere), the outputs are incomplete and this
+ *     call cannot report it -- it has returned before the kernel runs, and
+ *     the word that records the give-up is private to the library. Callers
+ *     that need that report use nvfp4_group_quantize (workspace word 1) or
+ *     nvfp4_group_quantize_graphsafe (status word).
  *   - Zeroing: each call zeroes the scratch (and row_amax, col_amax) on
  *     `stream` before its launch; nothing needs to start at zero.
  *   - Races: every call on a device shares the one scratch array, so calls

@@ -429,7 +429,11 @@ static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchWords
 constexpr int kMaxDevices = 64;
 
 // Device address of g_noalloc_scratch for the current device, looked up once
-// per device (with that device current) and cached. nullptr on failure.
+// per device (with that device current) and cached. nullptr on failure. The
+// address belongs to the device's context at lookup time; a cudaDeviceReset
+// of that device makes it stale (the header says so). A bounded wait that
+// gives up raises abort word 1 inside this array, which no call reads back:
+// HostRouting has no status word, so the give-up goes unreported here.
 uint32_t* noalloc_scratch() {
   static std::mutex mu;
   static uint32_t* addr[kMaxDevices] = {};

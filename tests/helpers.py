@@ -114,3 +114,54 @@ def gpu_quantize(x: torch.Tensor, m_splits, rows=True, cols=True, device="cuda",
     if cols:
         res["col_amax"] = ca.cpu().numpy()
     return res
+
+
+def host_threads() -> int:
+    """Cores this process may use (the oracle releases the GIL in its calls)."""
+    import os
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _eq_slice(got, want, what):
+    g = np.ascontiguousarray(got).reshape(-1).view(np.uint8)
+    w = np.ascontiguousarray(want).reshape(-1).view(np.uint8)
+    if g.shape != w.shape or not np.array_equal(g, w):
+        bad = np.nonzero(g != w)[0] if g.shape == w.shape else []
+        raise AssertionError(f"{what}: {len(bad)} bytes differ, first at {list(bad[:5])}")
+
+
+def check_groups_against_oracle(got: dict, xb: np.ndarray, m_splits, K: int, what: str = ""):
+    """Every byte of every group's outputs (row and column amax, rowwise and
+    colwise codes, scales and decode scales) against the oracle. A group's
+    outputs depend on its own rows only, so the oracle runs group by group,
+    spread over the host's cores; empty groups must have zero column amax and
+    decode scales. ``got`` holds the GPU's buffers cut at the routed rows."""
+    import concurrent.futures as cf
+    offs = workloads.row_offsets(m_splits)
+
+    def one(g):
+        m, o = m_splits[g], offs[g]
+        cs = slice(g * K, (g + 1) * K)
+        if m == 0:
+            assert np.all(got["col_amax"][cs] == 0) and np.all(got["col_s2"][cs] == 0), f"{what} empty g={g}"
+            return 0
+        sub = xb[o:o + m]
+        ra, ca = oracle.group_amax(sub, [m])
+        want = oracle.group_cast(sub, [m], ra, ca)
+        tag = f"{what} g={g}"
+        _eq_slice(got["row_amax"][o:o + m], ra, f"{tag} row_amax")
+        _eq_slice(got["col_amax"][cs], ca, f"{tag} col_amax")
+        for k in ("row_data", "row_scale", "row_s2"):
+            _eq_slice(got[k][o:o + m], want[k], f"{tag} {k}")
+        _eq_slice(got["col_data"][K * o // 2:K * (o + m) // 2], want["col_data"], f"{tag} col_data")
+        _eq_slice(got["col_scale"][K * o // 16:K * (o + m) // 16], want["col_scale"], f"{tag} col_scale")
+        _eq_slice(got["col_s2"][cs], want["col_s2"], f"{tag} col_s2")
+        return m
+
+    order = sorted(range(len(m_splits)), key=lambda g: -m_splits[g])  # largest first
+    with cf.ThreadPoolExecutor(max_workers=host_threads()) as ex:
+        done = sum(ex.map(one, order))
+    assert done == sum(m_splits)

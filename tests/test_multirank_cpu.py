@@ -66,7 +66,7 @@ def test_job_throughput_is_weak_scaling():
 def test_reference_arm_prints_on_rank_zero_only():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "3", "--tokens", "64"],
+                        "--gpus", "2", "--steps", "1", "--warmup", "3", "--tokens", "64"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
     env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
@@ -77,3 +77,32 @@ def test_reference_arm_prints_on_rank_zero_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "Gelem/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _env_without_ranks():
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "LOCAL_WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    return env
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` run as one process starts two ranks through
+    torch.distributed.run; rank 0 alone prints, and its line counts both.
+    (The reference arm needs no GPU, so the launcher runs here on the CPU.)"""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "3", "--tokens", "64"],
+                       env=_env_without_ranks(), capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+
+
+def test_gpus_flag_must_match_world_size():
+    env = dict(_env_without_ranks(), RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "1", "--steps", "1", "--warmup", "3", "--tokens", "64"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
