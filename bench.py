@@ -152,6 +152,13 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def wait_first(self, timeout: float = 10.0):
+        """Block until nvidia-smi has delivered a first sample (it can take a
+        few seconds to start), so that the timed region is sampled."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
     def _read(self):
         for ln in self.proc.stdout:
             self.lines.append(ln.strip())
@@ -423,7 +430,8 @@ def main():
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
     clocks.start()
-    time.sleep(0.3)
+    clocks.wait_first()
+    time.sleep(0.2)
     barrier()
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
@@ -438,7 +446,6 @@ def main():
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
     amax_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     cast_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
@@ -575,6 +582,10 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    # the sampler ran from just before the headline's timed region through
+    # every timed leg above (the headline region alone is ~10 ms, shorter than
+    # nvidia-smi's sampling interval)
+    clk = clocks.stop()
     # the downloaded bytes of the last step are the device's
     for k, v in outs[(e2e_steps - 1) % 2].items():
         if not torch.equal(host_out[k], v.cpu()):

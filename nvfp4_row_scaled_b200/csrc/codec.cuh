@@ -82,16 +82,28 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 
 namespace nvfp4rs {
 
-// E4M3 value table used by the block-scale shortcut below.
-// Table entry for E4M3 code c (0..127): {value, RN(1/value)}; codes 0 and
-// 0x7F (NaN, never produced by the saturating convert) hold {1, 0}.
-__device__ __forceinline__ float2 e4m3_entry(int c) {
-  if (c == 0 || c >= 0x7F) return make_float2(1.0f, 0.0f);
+// E4M3 tables used by the block-scale shortcut below, one entry per code c
+// (0..127): nv = -value(c) and r = RN(1/value(c)). Code 0 and 0x7F (NaN, never
+// produced by the saturating convert) hold nv = -1, r = 0, which makes the
+// element multiplier of a zero scale come out 0 with no branch.
+struct E4m3Table {
+  float nv[128];
+  float r[128];
+};
+
+// Entry c of the table, written by thread c of a block (c < 128).
+__device__ __forceinline__ void e4m3_table_fill(E4m3Table& tab, int c) {
+  if (c == 0 || c >= 0x7F) {
+    tab.nv[c] = -1.0f;
+    tab.r[c] = 0.0f;
+    return;
+  }
   const int e = c >> 3, m = c & 7;
   const float v = e == 0 ? __fmul_rn(static_cast<float>(m), 0x1p-9f)
                          : __uint_as_float((static_cast<uint32_t>(e + 120) << 23) |
                                            (static_cast<uint32_t>(m) << 20));
-  return make_float2(v, __frcp_rn(v));
+  tab.nv[c] = -v;
+  tab.r[c] = __frcp_rn(v);
 }
 
 }  // namespace nvfp4rs
@@ -126,6 +138,25 @@ __device__ __forceinline__ uint64_t mul2x(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+
+// pairwise a*b + c, one rounding per element
+__device__ __forceinline__ uint64_t fma2x(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// the low / high float of an f32x2 register pair
+__device__ __forceinline__ float lo_of(uint64_t p) {
+  float l;
+  asm("{.reg .b32 t;\n\tmov.b64 {%0, t}, %1;}" : "=f"(l) : "l"(p));
+  return l;
+}
+__device__ __forceinline__ float hi_of(uint64_t p) {
+  float h;
+  asm("{.reg .b32 t;\n\tmov.b64 {t, %0}, %1;}" : "=f"(h) : "l"(p));
+  return h;
 }
 
 // Codes of four pairs, pair i -> byte i with its low element in the low nibble.
@@ -192,24 +223,28 @@ __device__ __forceinline__ bool fast_path_amax(float a) {
   return a == 0.0f || (a >= kFastAmaxMin && a <= kFastAmaxMax);
 }
 
-__device__ __forceinline__ float div6_fast(float b) {
-  const float y = 0x1.555556p-3f;  // RN(1/6)
-  const float q0 = __fmul_rn(b, y);
-  const float r = __fmaf_rn(-q0, 6.0f, b);
-  return __fmaf_rn(r, y, q0);
-}
-
-__device__ __forceinline__ float elem_scale_fast(float S, float2 vy) {
-  const float q0 = __fmul_rn(S, vy.y);
-  const float r = __fmaf_rn(-q0, vy.x, S);
-  return fminf(__fmaf_rn(r, vy.y, q0), FLT_MAX);
-}
-
-__device__ __forceinline__ uint32_t scales2_fast(float bm0, float se0, float bm1, float se1,
-                                                 const float2* tab, float& enc0, float& enc1) {
-  const uint32_t p = e4m3x2(__fmul_rn(div6_fast(bm1), se1), __fmul_rn(div6_fast(bm0), se0));
-  enc0 = elem_scale_fast(se0, tab[p & 0xFFu]);
-  enc1 = elem_scale_fast(se1, tab[p >> 8]);
+// Two block scales at once (the blocks of one lane that share an f32x2
+// register pair): bm2 = {bmax0, bmax1} (block maxima), se2 = {S_enc0,
+// S_enc1}. Returns the two E4M3 codes (block 0 in bits 0..7, block 1 in bits
+// 8..15) and sets enc2 = {enc0, enc1}, the element multipliers:
+//   s32 = fl(fl(bmax/6) * S_enc), code = E4M3_rne_satfinite(s32),
+//   enc = fl(S_enc / e4m3(code)) (0 for a zero code).
+// Both divides use Markstein's correction with the reciprocal taken from
+// RN(1/6) or the table (tab.r), and the exact remainder fma(q0, -b, a) (the
+// table stores -value, so no negation is needed).
+__device__ __forceinline__ uint32_t scales2x_fast(uint64_t bm2, uint64_t se2, const E4m3Table& tab,
+                                                  uint64_t& enc2) {
+  const uint64_t y6 = pack2(0x1.555556p-3f, 0x1.555556p-3f);  // RN(1/6)
+  const uint64_t m6 = pack2(-6.0f, -6.0f);
+  const uint64_t q6 = mul2x(bm2, y6);
+  const uint64_t d6 = fma2x(fma2x(q6, m6, bm2), y6, q6);
+  const uint64_t s32 = mul2x(d6, se2);
+  const uint32_t p = e4m3x2(hi_of(s32), lo_of(s32));
+  const uint32_t c0 = p & 0xFFu, c1 = p >> 8;
+  const uint64_t nv = pack2(tab.nv[c0], tab.nv[c1]);
+  const uint64_t yr = pack2(tab.r[c0], tab.r[c1]);
+  const uint64_t q0 = mul2x(se2, yr);
+  enc2 = fma2x(fma2x(q0, nv, se2), yr, q0);
   return p;
 }
 
@@ -224,10 +259,15 @@ __device__ __forceinline__ uint32_t scales2_exact(float bm0, float se0, float bm
 }
 
 template <bool kExact>
-__device__ __forceinline__ uint32_t scales2_any(float bm0, float se0, float bm1, float se1,
-                                                const float2* tab, float& enc0, float& enc1) {
-  return kExact ? scales2_exact(bm0, se0, bm1, se1, enc0, enc1)
-                : scales2_fast(bm0, se0, bm1, se1, tab, enc0, enc1);
+__device__ __forceinline__ uint32_t scales2x_any(uint64_t bm2, uint64_t se2, const E4m3Table& tab,
+                                                 uint64_t& enc2) {
+  if (kExact) {
+    float e0, e1;
+    const uint32_t p = scales2_exact(lo_of(bm2), lo_of(se2), hi_of(bm2), hi_of(se2), e0, e1);
+    enc2 = pack2(e0, e1);
+    return p;
+  }
+  return scales2x_fast(bm2, se2, tab, enc2);
 }
 
 }  // namespace nvfp4rs

@@ -79,7 +79,7 @@ struct CastStage {
 // Dynamic shared memory of the cast kernel; `off` (E+1 int32) follows it.
 struct CastSmem {
   uint8_t tile[kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
-  float2 e4m3[128];                   // {value, RN(1/value)} per E4M3 code
+  E4m3Table e4m3;                     // the block-scale shortcut's E4M3 table
   float row_senc[kRows];
   float col_senc[kRows / kBlockRows][kCols];  // per 16-row block: [0] only, unless the tile is mixed
   uint64_t full[kStages];
@@ -277,10 +277,10 @@ struct StageColSink {
   }
 };
 
-// The shared tables a tile's encode reads: {value, RN(1/value)} of every
-// E4M3 code, and S_enc of the tile's 128 rows and 128 columns.
+// The shared tables a tile's encode reads: the E4M3 table of the block-scale
+// shortcut, and S_enc of the tile's 128 rows and 128 columns.
 struct EncodeTables {
-  const float2* e4m3;
+  const E4m3Table* e4m3;
   const float* row_senc;
   const float* col_senc;
 };
@@ -290,8 +290,9 @@ struct EncodeTables {
 // stores, the staging of the block scales (col_stg: [row block][column],
 // row_stg: [column block][row], both 128 wide) and the colwise codes handed
 // to col_sink. cc (0..15) is the lane's 8-column chunk of the tile, rb (0..7)
-// its 16-row block. kExact selects the IEEE-divide block scales (tiles with a
-// row or column amax outside the shortcut's range).
+// its 16-row block; the other half of each of its rowwise blocks is on lane
+// cc ^ 1 (the neighbouring lane). kExact selects the IEEE-divide block scales
+// (tiles with a row or column amax outside the shortcut's range).
 template <bool kExact, class ColSink>
 __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, uint8_t* col_stg,
                                              uint8_t* row_stg, bool do_row, bool do_col, int cc, int rb,
@@ -300,7 +301,7 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
   const bool odd = cc & 1;
 
   // ------------------------------------------------------ colwise scales
-  uint64_t cenc2[4];  // (enc of column 2q, enc of column 2q+1)
+  uint64_t cenc2[4];  // {enc of column 2q, enc of column 2q+1}
   if (do_col) {
     uint32_t m0 = v[0].x, m1 = v[0].y, m2 = v[0].z, m3 = v[0].w;
 #pragma unroll
@@ -312,54 +313,58 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
     }
     const uint32_t mw[4] = {m0 & 0x7FFF7FFFu, m1 & 0x7FFF7FFFu, m2 & 0x7FFF7FFFu,
                             m3 & 0x7FFF7FFFu};
-    const float* se = &tab.col_senc[8 * cc];
+    // the S_enc pair of columns (2q, 2q+1) is one aligned 8-byte entry
+    const uint64_t* se = reinterpret_cast<const uint64_t*>(&tab.col_senc[8 * cc]);
     uint32_t s8w[2] = {0u, 0u};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
-      float e0, e1;
-      const uint32_t p2 = scales2_any<kExact>(bf16lo(mw[q]), se[2 * q], bf16hi(mw[q]), se[2 * q + 1],
-                                              tab.e4m3, e0, e1);
-      cenc2[q] = pack2(e0, e1);
+      const uint32_t p2 = scales2x_any<kExact>(unpack2(mw[q]), se[q], *tab.e4m3, cenc2[q]);
       s8w[q >> 1] |= p2 << (16 * (q & 1));
     }
     *reinterpret_cast<uint2*>(&col_stg[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; q++) cenc2[q] = 0;
   }
 
   // ------------------------------------------------------ rowwise scales
   float renc[16];  // element multiplier of row i
   if (do_row) {
-    uint32_t P[8];  // (row 2k, row 2k+1) maxima over the whole 16-column block
+    uint32_t P[8];  // (row 2k, row 2k+1) maxima over the lane's 8 columns
 #pragma unroll
     for (int kk = 0; kk < 8; kk++) {
       const uint32_t a = maxabs2(maxabs2(v[2 * kk].x, v[2 * kk].y), maxabs2(v[2 * kk].z, v[2 * kk].w));
       const uint32_t b = maxabs2(maxabs2(v[2 * kk + 1].x, v[2 * kk + 1].y),
                                  maxabs2(v[2 * kk + 1].z, v[2 * kk + 1].w));
       P[kk] = maxabs2(prmt(a, b, 0x5410), prmt(a, b, 0x7632)) & 0x7FFF7FFFu;
-      P[kk] = umax2(P[kk], __shfl_xor_sync(0xFFFFFFFFu, P[kk], 1));
     }
-    // the even lane of a pair scales rows 0..7, the odd lane rows 8..15
-    float mine[8];
-    uint32_t s8mine[2] = {0u, 0u};
-    const float* rse = &tab.row_senc[rl + (odd ? 8 : 0)];
+    // The even lane of a pair scales rows 0..7, the odd lane rows 8..15: each
+    // sends the partner the half-block maxima of the partner's rows, and
+    // scales its own rows two at a time (row pairs are the f32x2 pairs).
+    const uint64_t* rse = reinterpret_cast<const uint64_t*>(&tab.row_senc[rl + (odd ? 8 : 0)]);
+    uint64_t mine[4];  // {enc of row 2k, of row 2k+1} of the lane's 8 rows
+    uint32_t s8w[2] = {0u, 0u};
 #pragma unroll
     for (int kk = 0; kk < 4; kk++) {
-      const uint32_t w = odd ? P[4 + kk] : P[kk];
-      const uint32_t p2 = scales2_any<kExact>(bf16lo(w), rse[2 * kk], bf16hi(w), rse[2 * kk + 1],
-                                              tab.e4m3, mine[2 * kk], mine[2 * kk + 1]);
-      s8mine[kk >> 1] |= p2 << (16 * (kk & 1));
+      const uint32_t send = odd ? P[kk] : P[kk + 4];
+      const uint32_t keep = odd ? P[kk + 4] : P[kk];
+      const uint32_t full = umax2(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 1));
+      const uint32_t p2 = scales2x_any<kExact>(unpack2(full), rse[kk], *tab.e4m3, mine[kk]);
+      s8w[kk >> 1] |= p2 << (16 * (kk & 1));
     }
+    *reinterpret_cast<uint2*>(&row_stg[(cc >> 1) * kRows + rl + (odd ? 8 : 0)]) = make_uint2(s8w[0], s8w[1]);
+    // rows 0..7's multipliers come from the even lane, rows 8..15's from the odd one
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int kk = 0; kk < 8; kk++) {
-      const float other = __shfl_xor_sync(0xFFFFFFFFu, mine[kk], 1);
-      renc[kk] = odd ? other : mine[kk];      // row kk
-      renc[8 + kk] = odd ? mine[kk] : other;  // row 8 + kk
+    for (int kk = 0; kk < 4; kk++) {
+      renc[2 * kk] = __shfl_sync(0xFFFFFFFFu, lo_of(mine[kk]), lane & ~1);
+      renc[2 * kk + 1] = __shfl_sync(0xFFFFFFFFu, hi_of(mine[kk]), lane & ~1);
+      renc[8 + 2 * kk] = __shfl_sync(0xFFFFFFFFu, lo_of(mine[kk]), lane | 1);
+      renc[9 + 2 * kk] = __shfl_sync(0xFFFFFFFFu, hi_of(mine[kk]), lane | 1);
     }
-    const uint32_t so0 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[0], 1);
-    const uint32_t so1 = __shfl_xor_sync(0xFFFFFFFFu, s8mine[1], 1);
-    if (!odd) {
-      *reinterpret_cast<uint4*>(&row_stg[(cc >> 1) * kRows + rl]) =
-          make_uint4(s8mine[0], s8mine[1], so0, so1);
-    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; i++) renc[i] = 0.0f;
   }
 
   // -------------------------------------------------------------- codes
@@ -579,7 +584,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
          i += static_cast<int64_t>(gridDim.x) * kCastThreads)
       gstore(&out.col_s2[i], s_dec_of(gload(&col_amax[i])));
   }
-  sm.e4m3[t] = e4m3_entry(t);
+  e4m3_table_fill(sm.e4m3, t);
 
   // this CTA's tiles: every gridDim-th of the row-major tile order
   const int n_ct = K >> 7;
@@ -676,7 +681,7 @@ group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant
 
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
                            : nullptr;
-    const EncodeTables tab{sm.e4m3, sm.row_senc, sm.col_senc[mixed ? rb : 0]};
+    const EncodeTables tab{&sm.e4m3, sm.row_senc, sm.col_senc[mixed ? rb : 0]};
     const bool row_store = kBlockRows * rb < valid;  // false past the routed rows
     if (slow_tile[k & 1])
       encode_patch<true>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);

@@ -54,7 +54,7 @@ struct alignas(16) PlainGroup {
 struct PlainSmem {
   uint8_t tile[kPGroups][kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
   PlainGroup grp[kPGroups];
-  float2 e4m3[128];
+  E4m3Table e4m3;
   RoutingSmem rs;
 };
 
@@ -138,7 +138,7 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
   const int t = threadIdx.x;
   const bool do_row = out.row_s2 != nullptr;
   const bool do_col = out.col_s2 != nullptr;
-  if (t < 128) sm.e4m3[t] = e4m3_entry(t);
+  if (t < 128) e4m3_table_fill(sm.e4m3, t);
 
   const int j = t / kCastThreads;  // warp group
   const int gt = t - j * kCastThreads;
@@ -176,11 +176,16 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
 
   int k = 0;
   bool failed = false;
+  // the tile's row and column tile, advanced by G tiles per step without a
+  // division; r0p, c0p: the previous tile's first row and column
+  const int Gq = G / n_ct, Gr = G - Gq * n_ct;
+  int rt = first / n_ct, ct = first - rt * n_ct;
+  int32_t r0p = 0;
+  int c0p = 0;
   for (int tl = first; tl < n_tiles; tl += G, k++) {
     const int s = k & 1;
     const int slot = k % kPSlots;
     const uint32_t phase = (k >> 1) & 1;
-    const int rt = tl / n_ct, ct = tl - rt * n_ct;
     const int32_t r0 = rt * kRows;
     const int c0 = ct * kCols;
     const bool ok = mbar_wait(&pg.full[s], phase);
@@ -216,12 +221,10 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       plain_issue(pg, sm.tile[j][s], &tmap, s, k + 2, tl + 2 * G, n_ct, rs, K, ra, ca);
     }
-    if (k >= 1) {  // the previous tile's staged scales (complete since the barrier)
-      const int tp = tl - G, rtp = tp / n_ct;
+    if (k >= 1)  // the previous tile's staged scales (complete since the barrier)
       store_scales<kTiled>(pg.col_scale[(k - 1) & 1], pg.row_scale[(k - 1) & 1], out, K,
-                           pg.info[(k - 1) % kPInfo][0], pg.info[(k - 1) % kPInfo][1], rtp * kRows,
-                           (tp - rtp * n_ct) * kCols, gt, do_row, do_col, keep);
-    }
+                           pg.info[(k - 1) % kPInfo][0], pg.info[(k - 1) % kPInfo][1], r0p, c0p, gt, do_row,
+                           do_col, keep);
     const int32_t o_g = pg.info[k % kPInfo][0];
     const size_t half_m = static_cast<size_t>(pg.info[k % kPInfo][1]) >> 1;
     uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc : nullptr;
@@ -229,21 +232,28 @@ group_cast_plain_kernel(const __grid_constant__ Routing routing, const __grid_co
                                     static_cast<size_t>(c0 + 8 * cc) * half_m + ((r0 - o_g + rl) >> 1)
                               : nullptr,
                        half_m, keep, {}};
-    const EncodeTables tab{sm.e4m3, pg.row_senc[slot], pg.col_senc[slot]};
+    const EncodeTables tab{&sm.e4m3, pg.row_senc[slot], pg.col_senc[slot]};
     if (any_slow)
       encode_patch<true>(v, tab, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst, row_pitch,
                          true, sink);
     else
       encode_patch<false>(v, tab, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst, row_pitch,
                           true, sink);
+    r0p = r0;
+    c0p = c0;
+    ct += Gr;
+    rt += Gq;
+    if (ct >= n_ct) {
+      ct -= n_ct;
+      rt++;
+    }
   }
 
   if (!failed && k >= 1) {  // the last tile's staged scales
     group_bar(bar_id);
-    const int tp = first + (k - 1) * G, rtp = tp / n_ct;
     store_scales<kTiled>(pg.col_scale[(k - 1) & 1], pg.row_scale[(k - 1) & 1], out, K,
-                         pg.info[(k - 1) % kPInfo][0], pg.info[(k - 1) % kPInfo][1], rtp * kRows,
-                         (tp - rtp * n_ct) * kCols, gt, do_row, do_col, keep);
+                         pg.info[(k - 1) % kPInfo][0], pg.info[(k - 1) % kPInfo][1], r0p, c0p, gt, do_row, do_col,
+                         keep);
   }
   if (failed && gt == 0) {
     // drain the loads this group issued and did not consume (tiles k, k+1)

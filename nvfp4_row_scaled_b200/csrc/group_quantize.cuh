@@ -210,7 +210,7 @@ struct alignas(16) QuantGroup {
 struct QuantSmem {
   uint8_t tile[kQGroups][kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
   QuantGroup grp[kQGroups];
-  float2 e4m3[128];                             // {value, RN(1/value)} per E4M3 code
+  E4m3Table e4m3;                               // the block-scale shortcut's E4M3 table
   RoutingSmem rs;
 };
 
@@ -385,7 +385,7 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
       if (off[g + 1] == off[g])
         for (int c = t; c < K; c += kQThreads) gstore(&out.col_s2[static_cast<size_t>(g) * K + c], s_dec_of(0.0f));
   }
-  if (t < 128) sm.e4m3[t] = e4m3_entry(t);
+  if (t < 128) e4m3_table_fill(sm.e4m3, t);
   if (t == 0) {
     for (int j = 0; j < kQGroups; j++) {
       QuantGroup& pg = sm.grp[j];
@@ -493,7 +493,7 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
                                       static_cast<size_t>(c0 + 8 * cc) * half_m + ((r0 - o_g + rl) >> 1)
                                 : nullptr,
                          half_m, once, {}};
-      const EncodeTables tab{sm.e4m3, pg.row_senc[s], pg.col_senc[s]};
+      const EncodeTables tab{&sm.e4m3, pg.row_senc[s], pg.col_senc[s]};
       if (any_slow)
         encode_patch<true>(v, tab, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
                            row_pitch, true, sink);
