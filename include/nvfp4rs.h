@@ -51,14 +51,18 @@
  *    CUDA launch returns NVFP4_ERR_CUDA. The graph-safe calls check the device
  *    routing on the device: a violation is written to *status_dev and the
  *    kernels write no output; they never trap and never hang.
- *  - Requirements (else NVFP4_ERR_UNSUPPORTED): K % 128 == 0, every group
- *    size m_g % 16 == 0 (the colwise block height; the one-launch calls
- *    need m_g % 128 == 0, the 128-row alignment of the grouped GEMM's scale
- *    layout), num_groups <= NVFP4_MAX_GROUPS, rows < 2^31, and every pointer
- *    16-byte aligned. Groups that are multiples of 128 rows take the fastest
- *    path; others are handled per 16-row block (a 128-row tile may then hold
- *    rows of several groups, and the last tile may be short). Inputs must be
- *    finite (a non-finite input gives unspecified codes, never a fault).
+ *  - Requirements: K % 16 == 0 (the rowwise block width; else
+ *    NVFP4_ERR_INVALID_ARG). Else NVFP4_ERR_UNSUPPORTED: every group size
+ *    m_g % 16 == 0 (the colwise block height), num_groups <=
+ *    NVFP4_MAX_GROUPS, rows < 2^31, and every pointer 16-byte aligned. The
+ *    one-launch calls, the MXFP4 calls and the 128x4-tiled scale layout also
+ *    need K % 128 == 0 and m_g % 128 == 0 (the 128-row alignment of the
+ *    grouped GEMM's scale layout). 128-row tiles inside one group on the
+ *    128-row grid, with K % 128 == 0, take the fastest path; the rest is
+ *    handled at the tile's edges in the same kernel (a 128-row tile may then
+ *    hold rows of several groups, the last row tile may be short, and the
+ *    last column tile partial). Inputs must be finite (a non-finite input
+ *    gives unspecified codes, never a fault).
  *  - Empty groups (m_g == 0) are allowed: their col_amax and col_s2 are 0
  *    and they own no bytes of col_data / col_scale.
  */
@@ -103,8 +107,8 @@ typedef enum {
                                  512 bytes each, in row-major tile order; scale (r, c) of
                                  a tile at byte (r % 32) * 16 + (r / 32) * 4 + c. Same
                                  sizes and per-group offsets as compact. Needs every
-                                 group to be a multiple of 128 rows (else
-                                 NVFP4_ERR_UNSUPPORTED). */
+                                 group to be a multiple of 128 rows and K % 128 == 0
+                                 (else NVFP4_ERR_UNSUPPORTED). */
 } nvfp4_scale_layout;
 
 /* Output buffers of the grouped cast (device pointers). A direction whose
@@ -190,10 +194,8 @@ NVFP4RS_API nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t 
  * Grouped cast, graph-safe routing: nvfp4_group_cast with the routing of
  * nvfp4_group_amax_graphsafe (same arguments, same status rules; status_dev
  * is reset to 0 by this call too). Byte-identical to nvfp4_group_cast for
- * equal routing. One memset of status and two launches: the kernel for
- * 128-aligned groups and the one for any groups, each of which checks the
- * device routing and returns at once unless it is the one to run (uniform
- * groups and tiled scales need only one).
+ * equal routing (the same kernel serves both). One memset of status and one
+ * launch, whatever the routing turns out to be on the device.
  */
 NVFP4RS_API nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
                                         const int64_t* first_dims_dev,
@@ -233,8 +235,8 @@ NVFP4RS_API size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, i
  *                   workspace must be ordered on one stream. After the call
  *                   word 1 is nonzero only if a bounded wait inside the kernel
  *                   gave up (not expected; the outputs are then incomplete).
- * Every group must be a multiple of 128 rows (else NVFP4_ERR_UNSUPPORTED);
- * for other group sizes use the two calls. With no direction requested
+ * Every group must be a multiple of 128 rows and K % 128 == 0 (else
+ * NVFP4_ERR_UNSUPPORTED); for other shapes use the two calls. With no direction requested
  * nothing is enqueued. Memsets of the workspace header, row_amax and
  * col_amax, then one launch.
  */

@@ -44,6 +44,7 @@ namespace nvfp4rs {
 namespace cg = cooperative_groups;
 
 constexpr int kAmaxThreads = 128;
+constexpr int kCols128 = 128;  // columns per chunk
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -66,9 +67,14 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
                   float* __restrict__ col_amax) {
   __shared__ RoutingSmem rs;
   __shared__ uint32_t rmax[kRows];
-  // dynamic: [K / cn] column maxima of this CTA, then the E+1 group offsets
+  // the cast launched after this kernel may start its set-up now
+  launch_dependents();
+  // dynamic: column maxima of this CTA's chunks (128 per chunk), then the
+  // E+1 group offsets. The ceil(K/128) chunks of 128 columns are dealt over
+  // the cluster; columns of the last chunk past K are neither read nor written.
+  const int cols = (((K + kCols128 - 1) / kCols128) / cn) * kCols128;
   extern __shared__ uint32_t cmax[];
-  routing.load(rs, reinterpret_cast<int32_t*>(cmax + K / cn));
+  routing.load(rs, reinterpret_cast<int32_t*>(cmax + cols));
 
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
@@ -77,7 +83,6 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   const int rank = static_cast<int>(cluster.block_rank());
   const int tile = blockIdx.x / cn;
   const int32_t r0 = tile * kRows;
-  const int cols = K / cn;
   const bool active = rs.ok && r0 < rs.total;
   // routed rows of the tile (a multiple of 16: the tail tile may be short),
   // this lane's 16-row block and its group; a tile that holds rows of more
@@ -100,12 +105,18 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
       // this lane: rows r0 + 16*rb + i (i < 16), columns c0 .. c0+7
       const int c_loc = (ch << 7) + (cc << 3);                // index into this CTA's cmax
       const int c_glb = ((ch * cn + rank) << 7) + (cc << 3);  // chunk ch of the CTA: rank + ch*cn
+      const bool col_ok = c_glb < K;                          // the lane's 8 columns are inside K
       // (a lane past the routed rows reads the tile's first block instead and
-      // contributes nothing)
+      // contributes nothing; a lane past K reads nothing)
       const uint4* p = x + (static_cast<size_t>(r0 + (lane_ok ? kBlockRows * rb : 0)) * K8) + (c_glb >> 3);
       uint4 v[16];
+      if (col_ok) {
 #pragma unroll
-      for (int i = 0; i < 16; i++) v[i] = ld_stream(p + i * K8);
+        for (int i = 0; i < 16; i++) v[i] = ld_stream(p + i * K8);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) v[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
 
       // column maxima over the lane's 16 rows
       uint32_t c0 = v[0].x, c1 = v[0].y, c2 = v[0].z, c3 = v[0].w;
@@ -157,7 +168,7 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
         atomicMax(&rmax[kBlockRows * rb + cc], rowm << 16);
       }
       if (mixed) {  // straight to this lane's group (a mixed tile is rare)
-        if (lane_ok && col_amax != nullptr) {
+        if (lane_ok && col_ok && col_amax != nullptr) {
           float* dst = col_amax + static_cast<size_t>(g_lane) * K + c_glb;
           const uint32_t w[4] = {c0 & 0x7FFF7FFFu, c1 & 0x7FFF7FFFu, c2 & 0x7FFF7FFFu, c3 & 0x7FFF7FFFu};
 #pragma unroll
@@ -184,8 +195,10 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   __syncthreads();
   if (active && !mixed && col_amax != nullptr) {
     float* dst = col_amax + static_cast<size_t>(g_first) * K;
-    for (int c = t; c < cols; c += kAmaxThreads)
-      red_max_u32(dst + ((((c >> 7) * cn + rank) << 7) | (c & 127)), cmax[c]);
+    for (int c = t; c < cols; c += kAmaxThreads) {
+      const int gc = (((c >> 7) * cn + rank) << 7) | (c & 127);
+      if (gc < K) red_max_u32(dst + gc, cmax[c]);
+    }
   }
   // every CTA of the cluster reaches both barriers, active or not
   cluster.sync();

@@ -8,40 +8,18 @@
 // scaling; TransformerEngine #3324 (row-scaled backward for GroupedLinear,
 // summary) adds the columnwise (transposed) operand with per-column amax.
 //
-// This file holds what both cast kernels share (TMA and mbarrier helpers,
-// the lane patch, encode_patch, the scale stores) and the general kernel for
-// groups that are multiples of 16 rows anywhere; the kernel for groups on the
-// 128-row grid is in group_cast_plain.cuh.
+// This file holds what the cast kernels share: TMA and mbarrier helpers, the
+// lane patch, the element and block-scale encoding (encode_codes,
+// encode_patch) and the scale stores. The grouped NVFP4 cast kernel is in
+// group_cast_plain.cuh, the one-launch amax + cast in group_quantize.cuh and
+// the MXFP4 cast in mx_cast.cuh.
 //
-// Structure of the general kernel (sm_100a):
-//  - Persistent CTAs (three per SM), each taking every gridDim-th 128 x 128
-//    tile of x in row-major tile order, so CTAs running at the same time read
-//    neighbouring tiles of the same rows. Group sizes are multiples of 16, so
-//    a lane's 16-row block lies in one group; a tile that a group boundary
-//    crosses ("mixed") keeps one column-scale table per 16-row block, and
-//    the last tile may hold fewer than 128 routed rows.
-//  - Tiles arrive by TMA: two 2-D tiled loads of 64 columns x 128 rows each
-//    (128-byte rows, 128-byte swizzle, no multicast, L2 evict-first) into a
-//    two-stage shared-memory ring, completion tracked by one mbarrier per
-//    stage. Once every thread holds its patch, the tile's stage is reused to
-//    stage that tile's outputs; it is refilled with the tile after next when
-//    those outputs have been stored.
-//  - Lane (cc, h) of warp w reads rows 32w + 16h + i (i < 16), columns
-//    8cc .. 8cc+7 of the tile from shared memory: a 16-row x 8-column patch in
-//    registers that holds 8 complete colwise blocks and 16 half rowwise blocks
-//    (completed with lane cc ^ 1). Both directions are encoded from it.
-//  - Block scales use exact shortcuts instead of IEEE divides: a per-CTA
-//    table of every E4M3 value and its correctly rounded reciprocal, and
-//    Markstein's correction (codec.cuh).
-//  - Outputs that are not contiguous per lane (colwise data and scales,
-//    rowwise scales) are staged in shared memory and stored as full 8- or
-//    16-byte pieces of contiguous runs, with an L2 evict-last hint: a group's
-//    transposed outputs and the 8-byte scale pieces fill their sectors from
-//    several tiles, and should meet in L2 before being written back.
-// Tiles of groups that are not multiples of 128 rows, mixed tiles and the
-// short last tile store their colwise outputs per 16-row block
-// (store_staged_general). Every CTA also writes a slice of
-// col_s2 = S_dec(col_amax) (all E*K entries, empty groups included).
+// The lane patch (all kernels): a lane holds 16 rows x 8 columns of a
+// 128 x 128 tile in registers -- 8 complete colwise blocks and 16 half
+// rowwise blocks, completed with the neighbouring lane -- and encodes both
+// directions from it. Block scales use exact shortcuts instead of IEEE
+// divides: a per-CTA table of every E4M3 value and its correctly rounded
+// reciprocal, and Markstein's correction (codec.cuh).
 #pragma once
 
 #include <cuda.h>
@@ -76,12 +54,9 @@ struct CastStage {
   uint8_t row_scale[8 * kRows];  // [column block][row]
 };
 
-// Dynamic shared memory of the cast kernel; `off` (E+1 int32) follows it.
+// Dynamic shared memory of the MXFP4 cast kernel; `off` (E+1 int32) follows it.
 struct CastSmem {
   uint8_t tile[kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
-  E4m3Table e4m3;                     // the block-scale shortcut's E4M3 table
-  float row_senc[kRows];
-  float col_senc[kRows / kBlockRows][kCols];  // per 16-row block: [0] only, unless the tile is mixed
   uint64_t full[kStages];
 };
 
@@ -278,12 +253,19 @@ struct StageColSink {
 };
 
 // The shared tables a tile's encode reads: the E4M3 table of the block-scale
-// shortcut, and S_enc of the tile's 128 rows and 128 columns.
+// shortcut, and S_enc of the tile's 128 rows.
 struct EncodeTables {
   const E4m3Table* e4m3;
   const float* row_senc;
-  const float* col_senc;
 };
+
+// S_enc of the lane's 8 columns as four pairs (2q, 2q+1), from a 128-entry
+// table of the tile's columns.
+__device__ __forceinline__ void col_senc_pairs(const float* col_senc, int cc, uint64_t (&cse)[4]) {
+  const uint64_t* se = reinterpret_cast<const uint64_t*>(&col_senc[8 * cc]);
+#pragma unroll
+  for (int q = 0; q < 4; q++) cse[q] = se[q];
+}
 
 // Everything one lane does for one tile after its 16 x 8 patch is in
 // registers: block scales of both directions, all codes, the rowwise data
@@ -291,12 +273,14 @@ struct EncodeTables {
 // row_stg: [column block][row], both 128 wide) and the colwise codes handed
 // to col_sink. cc (0..15) is the lane's 8-column chunk of the tile, rb (0..7)
 // its 16-row block; the other half of each of its rowwise blocks is on lane
-// cc ^ 1 (the neighbouring lane). kExact selects the IEEE-divide block scales
-// (tiles with a row or column amax outside the shortcut's range).
+// cc ^ 1 (the neighbouring lane). cse: S_enc of the lane's 8 columns in
+// pairs (2q, 2q+1). kExact selects the IEEE-divide block scales (tiles with a
+// row or column amax outside the shortcut's range).
 template <bool kExact, class ColSink>
-__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, uint8_t* col_stg,
-                                             uint8_t* row_stg, bool do_row, bool do_col, int cc, int rb,
-                                             uint8_t* rdst, size_t row_pitch, bool row_store, ColSink&& col_sink) {
+__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, const uint64_t (&cse)[4],
+                                             uint8_t* col_stg, uint8_t* row_stg, bool do_row, bool do_col, int cc,
+                                             int rb, uint8_t* rdst, size_t row_pitch, bool row_store,
+                                             ColSink&& col_sink) {
   const int rl = 16 * rb;
   const bool odd = cc & 1;
 
@@ -313,12 +297,10 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
     }
     const uint32_t mw[4] = {m0 & 0x7FFF7FFFu, m1 & 0x7FFF7FFFu, m2 & 0x7FFF7FFFu,
                             m3 & 0x7FFF7FFFu};
-    // the S_enc pair of columns (2q, 2q+1) is one aligned 8-byte entry
-    const uint64_t* se = reinterpret_cast<const uint64_t*>(&tab.col_senc[8 * cc]);
     uint32_t s8w[2] = {0u, 0u};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
-      const uint32_t p2 = scales2x_any<kExact>(unpack2(mw[q]), se[q], *tab.e4m3, cenc2[q]);
+      const uint32_t p2 = scales2x_any<kExact>(unpack2(mw[q]), cse[q], *tab.e4m3, cenc2[q]);
       s8w[q >> 1] |= p2 << (16 * (q & 1));
     }
     *reinterpret_cast<uint2*>(&col_stg[rb * kCols + 8 * cc]) = make_uint2(s8w[0], s8w[1]);
@@ -369,15 +351,6 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
 
   // -------------------------------------------------------------- codes
   encode_codes(v, renc, cenc2, do_row, do_col, rdst, row_pitch, row_store, col_sink);
-}
-
-// encode_patch with every output but the rowwise data staged in st.
-template <bool kExact>
-__device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, CastStage& st,
-                                             bool do_row, bool do_col, int cc, int rb,
-                                             uint8_t* rdst, size_t row_pitch, bool row_store = true) {
-  encode_patch<kExact>(v, tab, st.col_scale, st.row_scale, do_row, do_col, cc, rb, rdst, row_pitch, row_store,
-                       StageColSink{st, cc, rb});
 }
 
 // The 128x4-tiled scale layout (the grouped GEMM's swizzle contract; see the
@@ -464,253 +437,6 @@ __device__ __forceinline__ void store_scales(const uint8_t* col_stg, const uint8
       st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
                         make_uint2(s0, s1), keep);
     }
-  }
-}
-
-// Everything a tile of a 128-aligned group staged in st: colwise data, then
-// the block scales.
-template <bool kTiled>
-__device__ __forceinline__ void store_staged(const CastStage& st, const CastOut& out, int K,
-                                             int32_t o_g, int64_t m_g, int32_t r0, int c0, int t,
-                                             bool do_row, bool do_col, uint64_t keep) {
-  if (do_col) store_col_data(st, out.col_data, K, o_g, m_g, r0, c0, t, keep);
-  store_scales<kTiled>(st.col_scale, st.row_scale, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
-}
-
-// A whole tile of one group that is not on the 128-row grid: colwise codes
-// as 8-byte pieces (the runs are 8-byte aligned), colwise scales as bytes.
-__device__ __forceinline__ void store_staged_single(const CastStage& st, const CastOut& out, int K, int32_t o_g,
-                                                    int64_t m_g, int32_t r0, int c0, int t, bool do_row,
-                                                    bool do_col, uint64_t keep) {
-  if (do_col) {
-    const size_t half_m = static_cast<size_t>(m_g) >> 1, m16 = static_cast<size_t>(m_g) >> 4;
-    uint8_t* gd = out.col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
-    uint8_t* gs = out.col_scale + (static_cast<size_t>(K) * o_g >> 4) + ((r0 - o_g) >> 4);
-#pragma unroll
-    for (int kk = 0; kk < 8; kk++) {
-      const int u = kk * kCastThreads + t;
-      const int col = u >> 3, b = u & 7;
-      const int sw = (col >> 3) & 7;
-      st_global_u2_hint(gd + static_cast<size_t>(c0 + col) * half_m + 8 * b,
-                        *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * (b ^ sw)]), keep);
-      gstore(&gs[static_cast<size_t>(c0 + col) * m16 + b], st.col_scale[b * kCols + col]);
-    }
-  }
-  if (do_row) {
-    uint32_t s0 = 0u, s1 = 0u;
-#pragma unroll
-    for (int r = 0; r < 4; r++) {
-      s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
-      s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
-    }
-    st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4), make_uint2(s0, s1), keep);
-  }
-}
-
-// (Never sees tiled scales: those need 128-aligned groups, whose tiles are
-// all plain.) Stores of a tile that store_staged cannot take: a tile crossing a group
-// boundary, the short last tile, or a group that does not start and end on
-// 128-row boundaries (its colwise runs are then only 8-byte aligned). Colwise outputs go
-// per (column, 16-row block): 8 bytes of codes and one scale byte, to the
-// block's own group; only blocks of routed rows (16 * b < valid) are stored.
-// `g` is the tile's group when it holds one group only (mixed == false).
-__device__ __noinline__ void store_staged_general(const CastStage& st, const CastOut& out,
-                                                     const RoutingSmem& rs, int K, int32_t r0, int c0,
-                                                     int t, int valid, bool mixed, int g, bool do_row,
-                                                     bool do_col, uint64_t keep) {
-  // thread t always stores 16-row block t % 8 (of columns t / 8 + 16 kk)
-  const int b = t & 7;
-  if (do_col && kBlockRows * b < valid) {
-    const int32_t r = r0 + kBlockRows * b;
-    const int gb = mixed ? group_of_row(rs, r) : g;
-    const int32_t o = rs.off[gb];
-    const size_t m = static_cast<size_t>(rs.off[gb + 1] - o);
-#pragma unroll 2
-    for (int kk = 0; kk < 8; kk++) {
-      const int col = (kk * kCastThreads + t) >> 3;
-      const int sw = (col >> 3) & 7;
-      const uint2 d = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * (b ^ sw)]);
-      st_global_u2_hint(out.col_data + (static_cast<size_t>(K) * o >> 1) + static_cast<size_t>(c0 + col) * (m >> 1) +
-                            ((r - o) >> 1),
-                        d, keep);
-      gstore(&out.col_scale[(static_cast<size_t>(K) * o >> 4) + static_cast<size_t>(c0 + col) * (m >> 4) + ((r - o) >> 4)],
-             st.col_scale[b * kCols + col]);
-    }
-  }
-  if (do_row && t < valid) {
-    uint32_t s0 = 0u, s1 = 0u;
-#pragma unroll
-    for (int r = 0; r < 4; r++) {
-      s0 |= static_cast<uint32_t>(st.row_scale[r * kRows + t]) << (8 * r);
-      s1 |= static_cast<uint32_t>(st.row_scale[(r + 4) * kRows + t]) << (8 * r);
-    }
-    st_global_u2_hint(out.row_scale + static_cast<size_t>(r0 + t) * (K >> 4) + (c0 >> 4),
-                      make_uint2(s0, s1), keep);
-  }
-}
-
-// ------------------------------------------------------------------ kernel
-
-// The general cast: groups that are multiples of 16 rows anywhere (the
-// 128-aligned case runs group_cast_plain_kernel). A tile may cross group
-// boundaries (mixed: one column-scale table per 16-row block) and the last
-// row tile may be short.
-template <class Routing>
-__global__ void __launch_bounds__(kCastThreads, 3)
-group_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ CUtensorMap tmap,
-                  int32_t K, const float* __restrict__ row_amax,
-                  const float* __restrict__ col_amax, const CastOut out) {
-  // the 128-byte swizzle wants each stage 1024-byte aligned; the host adds
-  // 1024 bytes of slack for this
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  CastSmem& sm = *reinterpret_cast<CastSmem*>(base);
-  int32_t* off = reinterpret_cast<int32_t*>(base + ((sizeof(CastSmem) + 15) & ~size_t{15}));
-  __shared__ RoutingSmem rs;
-  __shared__ int slow_tile[2];  // per-tile flag (alternating): some amax outside the shortcut range
-
-  routing.load(rs, off);
-  if (!rs.ok) return;
-
-  const int t = threadIdx.x;
-  // a requested direction always has its decode-scale buffer (the data and
-  // scale buffers may be NULL only when there are no rows)
-  const bool do_row = out.row_s2 != nullptr;
-  const bool do_col = out.col_s2 != nullptr;
-
-  if (do_col) {  // decode scales of all columns of all groups, spread over the grid
-    const int64_t n = static_cast<int64_t>(rs.E) * K;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kCastThreads + t; i < n;
-         i += static_cast<int64_t>(gridDim.x) * kCastThreads)
-      gstore(&out.col_s2[i], s_dec_of(gload(&col_amax[i])));
-  }
-  e4m3_table_fill(sm.e4m3, t);
-
-  // this CTA's tiles: every gridDim-th of the row-major tile order
-  const int n_ct = K >> 7;
-  const int n_tiles = ((rs.total + kRows - 1) >> 7) * n_ct;  // the last row tile may be short
-  const int G = gridDim.x;
-  if (t == 0) {
-    for (int s = 0; s < kStages; s++) mbar_init(&sm.full[s], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    slow_tile[0] = 0;
-    slow_tile[1] = 0;
-  }
-  __syncthreads();
-  if (t == 0)
-    for (int s = 0; s < kStages && blockIdx.x + s * G < n_tiles; s++) issue_tile(sm, &tmap, s, blockIdx.x + s * G, n_ct);
-
-  const int lane = t & 31, warp = t >> 5;
-  const int cc = lane & 15, h = lane >> 4;
-  const int rb = 2 * warp + h;  // 16-row block of the tile, 0..7
-  const int rl = 16 * rb;       // first tile row of this lane
-  const size_t row_pitch = static_cast<size_t>(K) >> 1;
-
-  int k = 0;
-  bool failed = false;
-  int cur_rt = -1;
-  bool row_slow = false;
-  int g = 0;  // group of the row tile's first row
-  int32_t o_g = 0;
-  int64_t m_g = 0;
-  const uint64_t keep = policy_evict_last();
-  for (int tl = blockIdx.x; tl < n_tiles; tl += G, k++) {
-    const int s = k % kStages;
-    const uint32_t phase = (k / kStages) & 1;
-    const int rt = tl / n_ct, ct = tl - rt * n_ct;
-    const int32_t r0 = rt * kRows;
-    const int c0 = ct * kCols;
-    if (t == 0) slow_tile[(k + 1) & 1] = 0;  // flag of the next tile (last read a tile ago)
-    bool slow = false;
-    const int valid = min(kRows, rs.total - r0);  // routed rows (a multiple of 16)
-    if (rt != cur_rt) {  // new row tile: its group(s) and its rows' encode scales
-      cur_rt = rt;
-      g = group_of_row(rs, r0);
-      o_g = rs.off[g];
-      m_g = rs.off[g + 1] - o_g;
-      if (do_row) {
-        const bool in = t < valid;
-        const float a = in ? gload(&row_amax[r0 + t]) : 0.0f;
-        sm.row_senc[t] = s_enc_of(a);
-        row_slow = in && !fast_path_amax(a);
-        if (ct == 0 && in) gstore(&out.row_s2[r0 + t], s_dec_of(a));
-      }
-    }
-    slow |= row_slow;
-    const bool mixed = o_g + m_g < r0 + valid;  // the tile crosses a group boundary
-    if (do_col) {
-      if (!mixed) {
-        const float a = gload(&col_amax[static_cast<size_t>(g) * K + c0 + t]);
-        sm.col_senc[0][t] = s_enc_of(a);
-        slow |= !fast_path_amax(a);
-      } else {  // one column table per 16-row block, from the block's group
-        int gb = g, gprev = -1;
-        float e = 1.0f;
-        for (int b = 0; kBlockRows * b < valid; b++) {
-          while (rs.off[gb + 1] <= r0 + kBlockRows * b) gb++;  // groups only move forward
-          if (gb != gprev) {  // a new group (a tile holds few): its column scale
-            const float a = gload(&col_amax[static_cast<size_t>(gb) * K + c0 + t]);
-            e = s_enc_of(a);
-            slow |= !fast_path_amax(a);
-            gprev = gb;
-          }
-          sm.col_senc[b][t] = e;
-        }
-      }
-    }
-    if (slow) slow_tile[k & 1] = 1;
-
-    // this lane's 16 x 8 patch from the swizzled stage
-    const bool ok = mbar_wait(&sm.full[s], phase);
-    uint4 v[16];
-    load_patch(sm.tile[s], cc, rl, v);
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
-    // The other stage held tile k-1, whose staged outputs were stored before
-    // this barrier: refill it with tile k+1 (tiles 0 and 1 came in the prologue).
-    // (issued by lane 0 of warp k % 4, so that the issue work does not always
-    // delay the same warp at the next barrier)
-    if (t == 32 * (k & 3) && k >= 1 && tl + G < n_tiles) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_tile(sm, &tmap, (k + 1) % kStages, tl + G, n_ct);
-    }
-    // stage s is free once every thread holds its patch: it stages the outputs
-    CastStage& st = *reinterpret_cast<CastStage*>(sm.tile[s]);
-
-    uint8_t* rdst = do_row ? out.row_data + static_cast<size_t>(r0 + rl) * row_pitch + (c0 >> 1) + 4 * cc
-                           : nullptr;
-    const EncodeTables tab{&sm.e4m3, sm.row_senc, sm.col_senc[mixed ? rb : 0]};
-    const bool row_store = kBlockRows * rb < valid;  // false past the routed rows
-    if (slow_tile[k & 1])
-      encode_patch<true>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
-    else
-      encode_patch<false>(v, tab, st, do_row, do_col, cc, rb, rdst, row_pitch, row_store);
-    __syncthreads();
-    // (the tile's shape again, rather than kept live through the encode) A
-    // whole tile of a group that starts and ends on 128-row boundaries takes
-    // store_staged, whose 16-byte colwise data and 8-byte colwise scale stores
-    // need those boundaries; a whole tile of one group otherwise,
-    // store_staged_single; every other tile, store_staged_general.
-    {
-      const int valid2 = min(kRows, rs.total - r0);
-      const bool mixed2 = o_g + m_g < r0 + valid2;
-      if (!mixed2 && valid2 == kRows && ((o_g | m_g) & (kRows - 1)) == 0)
-        store_staged<false>(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
-      else if (!mixed2 && valid2 == kRows)
-        store_staged_single(st, out, K, o_g, m_g, r0, c0, t, do_row, do_col, keep);
-      else
-        store_staged_general(st, out, rs, K, r0, c0, t, valid2, mixed2, g, do_row, do_col, keep);
-    }
-  }
-
-  if (failed && t == 0) {
-    // drain the loads this CTA issued and did not consume (tile k, and tile 1
-    // when the prologue's second load is still outstanding), then report
-    for (int j = k; j <= (k == 0 ? 1 : k) && blockIdx.x + j * G < n_tiles; j++)
-      mbar_wait(&sm.full[j % kStages], (j / kStages) & 1);
-    routing.report(NVFP4_ERR_TIMEOUT);
   }
 }
 

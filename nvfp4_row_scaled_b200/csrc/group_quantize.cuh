@@ -492,13 +492,15 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
       DirectColSink sink{do_col ? out.col_data + (static_cast<size_t>(K) * o_g >> 1) +
                                       static_cast<size_t>(c0 + 8 * cc) * half_m + ((r0 - o_g + rl) >> 1)
                                 : nullptr,
-                         half_m, once, {}};
-      const EncodeTables tab{&sm.e4m3, pg.row_senc[s], pg.col_senc[s]};
+                         half_m, once, do_col, {}};
+      const EncodeTables tab{&sm.e4m3, pg.row_senc[s]};
+      uint64_t cse[4];
+      if (do_col) col_senc_pairs(pg.col_senc[s], cc, cse);
       if (any_slow)
-        encode_patch<true>(v, tab, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
+        encode_patch<true>(v, tab, cse, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
                            row_pitch, true, sink);
       else
-        encode_patch<false>(v, tab, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
+        encode_patch<false>(v, tab, cse, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
                             row_pitch, true, sink);
     } else {
       // ------------------------------------------------------------ A item

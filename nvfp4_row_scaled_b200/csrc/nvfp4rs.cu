@@ -85,14 +85,14 @@ struct SpanList {
 #endif
 
 // CTAs per cluster along K for the amax kernel: the largest d <= 8 that
-// divides the number of 128-column chunks and leaves every CTA at least 4 of
-// them -- below that the per-CTA setup (routing, the cluster merge of the
+// divides the number of 128-column chunks (ceil(K/128)) and leaves every CTA
+// at least 4 of them -- below that the per-CTA setup (routing, the cluster merge of the
 // row maxima) costs more than the extra CTAs gain: at K = 2048, 4 CTAs of 4
 // chunks run the amax 9-15% faster than 8 CTAs of 2. A problem that would
 // then have fewer CTAs than the GPU has SMs takes the largest d <= 8 that
 // divides the chunks instead.
 int amax_cluster(int64_t K, int64_t tiles = INT64_MAX, int sms = 0) {
-  const int64_t chunks = K / kCols;
+  const int64_t chunks = (K + kCols - 1) / kCols;
   int widest = 1, wide4 = 1;
   for (int d = 8; d > 1; d--)
     if (chunks % d == 0) {
@@ -102,14 +102,20 @@ int amax_cluster(int64_t K, int64_t tiles = INT64_MAX, int sms = 0) {
   return (sms > 0 && tiles < (sms + wide4 - 1) / wide4) ? widest : wide4;
 }
 
-// Shape checks shared by both steps and both routings.
-nvfp4_status check_shape(const void* x, int64_t rows, int64_t K, int32_t E) {
+// Columns of the amax kernel's per-CTA table: its share of the 128-column chunks.
+int64_t amax_cta_cols(int64_t K, int cn) { return ((K + kCols - 1) / kCols) / cn * kCols; }
+
+// Shape checks shared by both steps and both routings: K any multiple of 16
+// (k128: the calls that need K % 128 == 0 -- the one-launch, MXFP4 and
+// tiled-scale paths -- return NVFP4_ERR_UNSUPPORTED otherwise).
+nvfp4_status check_shape(const void* x, int64_t rows, int64_t K, int32_t E, bool k128 = false) {
   if (rows < 0 || K < 0 || E < 0) return NVFP4_ERR_INVALID_ARG;
   if (K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && x == nullptr) return NVFP4_ERR_INVALID_ARG;
-  if (K % kCols != 0 || E > NVFP4_MAX_GROUPS || rows > kMaxRows) return NVFP4_ERR_UNSUPPORTED;
-  if (K / amax_cluster(K) > kMaxAmaxCols) return NVFP4_ERR_UNSUPPORTED;
-  if ((rows / kRows) * (K / kCols) > (int64_t{1} << 30)) return NVFP4_ERR_UNSUPPORTED;  // tile ids fit int32
+  if ((k128 && K % kCols != 0) || E > NVFP4_MAX_GROUPS || rows > kMaxRows) return NVFP4_ERR_UNSUPPORTED;
+  if (amax_cta_cols(K, amax_cluster(K)) > kMaxAmaxCols) return NVFP4_ERR_UNSUPPORTED;
+  if (((rows + kRows - 1) / kRows) * ((K + kCols - 1) / kCols) > (int64_t{1} << 30))
+    return NVFP4_ERR_UNSUPPORTED;  // tile ids fit int32
   if (!aligned(x, 16)) return NVFP4_ERR_UNSUPPORTED;
   return NVFP4_OK;
 }
@@ -133,10 +139,10 @@ nvfp4_status host_routing(const int64_t* m_splits, int32_t E, int64_t sum_M, Hos
   }
   if (total != sum_M) return NVFP4_ERR_INVALID_ARG;
   if (unaligned) return NVFP4_ERR_UNSUPPORTED;
-  if (all_128 != nullptr) {
-    *all_128 = true;
-    for (int32_t g = 0; g < E; g++) *all_128 = *all_128 && m_splits[g] % kRows == 0;
-  }
+  bool a128 = true;
+  for (int32_t g = 0; g < E; g++) a128 = a128 && m_splits[g] % kRows == 0;
+  if (all_128 != nullptr) *all_128 = a128;
+  r.all128 = a128;
   r.total = static_cast<int32_t>(total);
   return NVFP4_OK;
 }
@@ -161,7 +167,7 @@ nvfp4_status device_routing(const int64_t* first_dims, const int64_t* offsets, i
     return NVFP4_ERR_INVALID_ARG;
   }
   if (!aligned(status, 4) || !aligned(first_dims, 8) || !aligned(offsets, 8)) return NVFP4_ERR_UNSUPPORTED;
-  r = DeviceRouting{first_dims, offsets, status, K, capacity_rows, E, align, m, 0};
+  r = DeviceRouting{first_dims, offsets, status, K, capacity_rows, E, align, m};
   return NVFP4_OK;
 }
 
@@ -204,7 +210,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 // 128-byte swizzle (the layout the cast kernel reads back).
 bool x_tensor_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K) {
   std::memset(map, 0, sizeof(*map));
-  if (rows == 0 || K < kCols) return true;  // no tile: the map is never used
+  if (rows == 0 || K == 0) return true;  // no tile: the map is never used
   PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
@@ -232,7 +238,7 @@ nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t rows, in
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return NVFP4_ERR_CUDA;
   const int cn = amax_cluster(K, tiles, sms);
-  const size_t smem = static_cast<size_t>(K / cn) * sizeof(uint32_t) + sizeof(int32_t) * (E + 1);
+  const size_t smem = static_cast<size_t>(amax_cta_cols(K, cn)) * sizeof(uint32_t) + sizeof(int32_t) * (E + 1);
   auto kernel = group_amax_kernel<Routing>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -256,35 +262,31 @@ nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t rows, in
                                         row_amax, col_amax));
 }
 
-// general: some group may not start and end on 128-row boundaries (always
-// so for device routing, which the host cannot see).
+// The cast kernel: one CTA per SM, three warp groups, for every routing
+// (groups of any multiple of 16 rows; general tiles take the kernel's edge
+// path, see group_cast_plain.cuh).
 template <class Routing>
 nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
                          const float* row_amax, const float* col_amax, const nvfp4_outputs* out,
-                         bool do_col, bool general, cudaStream_t stream) {
-  const int64_t tiles = ((rows + kRows - 1) / kRows) * (K / kCols);
+                         bool do_col, cudaStream_t stream) {
+  const int64_t tiles = ((rows + kRows - 1) / kRows) * ((K + kCols - 1) / kCols);
   const bool s2_work = do_col && E > 0 && K > 0;
   if (tiles == 0 && !s2_work) return NVFP4_OK;
   CUtensorMap map;
   if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
-  // tiled scales come with 128-row groups only (checked on the host, or on
-  // the device by the routing): those run the plain kernel
+  // tiled scales come with 128-row groups and K % 128 == 0 only (checked on
+  // the host, or on the device by the routing): every tile is plain
   const bool tiled = out->scale_layout == NVFP4_SCALE_TILED_128X4;
-  // the plain kernel: one CTA per SM, three warp groups; the general one:
-  // as many 4-warp CTAs as fit
-  auto kernel = general ? group_cast_kernel<Routing>
-                        : (tiled ? group_cast_plain_kernel<Routing, true> : group_cast_plain_kernel<Routing, false>);
-  const int threads = general ? kCastThreads : kPThreads;
-  const int64_t units = general ? tiles : (tiles + kPGroups - 1) / kPGroups;
-  // + room to align the block to 1024 bytes
-  const size_t smem = (general ? cast_smem_bytes(E) : plain_smem_bytes(E)) + 1024;
+  auto kernel = tiled ? group_cast_plain_kernel<Routing, true> : group_cast_plain_kernel<Routing, false>;
+  const int64_t units = (tiles + kPGroups - 1) / kPGroups;
+  const size_t smem = plain_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPThreads, smem) != cudaSuccess)
     return NVFP4_ERR_CUDA;
   if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
@@ -301,9 +303,17 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
                   .set(stream));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(threads);
+  cfg.blockDim = dim3(kPThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  // programmatic dependent launch: the kernel's set-up may overlap the tail
+  // of the kernel before it (the grouped amax); it waits for that kernel
+  // before reading anything (griddepcontrol.wait, group_cast_plain.cuh)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), row_amax,
                                         col_amax, o));
 }
@@ -574,9 +584,9 @@ nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int64_t K,
   bool all_128 = true;
   s = host_routing(m_splits_host, num_groups, sum_M, routing, kBlockRows, &all_128);
   if (s != NVFP4_OK) return s;
-  if (out->scale_layout == NVFP4_SCALE_TILED_128X4 && !all_128) return NVFP4_ERR_UNSUPPORTED;
-  return launch_cast(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, out, do_col, !all_128,
-                     stream);
+  // the 128x4-tiled layout is made of whole 128-row, 4-block tiles
+  if (out->scale_layout == NVFP4_SCALE_TILED_128X4 && (!all_128 || K % kCols != 0)) return NVFP4_ERR_UNSUPPORTED;
+  return launch_cast(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, out, do_col, stream);
 }
 
 nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
@@ -618,30 +628,17 @@ nvfp4_status nvfp4_group_cast_graphsafe(const void* x_bf16, int64_t capacity_row
       (do_col && num_groups > 0 && K > 0 && col_amax == nullptr))
     return NVFP4_ERR_INVALID_ARG;
   if (!aligned(row_amax, 16) || !aligned(col_amax, 16)) return NVFP4_ERR_UNSUPPORTED;
-  DeviceRouting routing;  // tiled scales need 128-row groups: checked on the device
+  // tiled scales need 128-row groups (checked on the device) and K % 128 == 0
+  const bool tiled = out->scale_layout == NVFP4_SCALE_TILED_128X4;
+  if (tiled && K % kCols != 0) return NVFP4_ERR_UNSUPPORTED;
+  DeviceRouting routing;
   s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups,
-                     out->scale_layout == NVFP4_SCALE_TILED_128X4 ? kRows : kBlockRows, routing);
+                     tiled ? kRows : kBlockRows, routing);
   if (s != NVFP4_OK) return s;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK) return s;
   if (K == 0) return NVFP4_OK;
-  if (out->scale_layout == NVFP4_SCALE_TILED_128X4)  // 128-row groups only: every tile is plain
-    return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
-                       /*general=*/false, stream);
-  if (routing.uniform_rows >= 0)
-    return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
-                       routing.uniform_rows % kRows != 0, stream);
-  // The host cannot see whether the groups are 128-aligned: enqueue the plain
-  // instantiation, which runs only if they all are, and the general one,
-  // which runs only if some are not (the other exits after the routing).
-  DeviceRouting plain = routing, general = routing;
-  plain.only_128 = 1;
-  general.only_128 = -1;
-  s = launch_cast(plain, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
-                  /*general=*/false, stream);
-  if (s != NVFP4_OK) return s;
-  return launch_cast(general, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col,
-                     /*general=*/true, stream);
+  return launch_cast(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, out, do_col, stream);
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* scale, const float* s2,
@@ -663,7 +660,7 @@ nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
                                   const int64_t* m_splits_host, int32_t num_groups, float* row_amax,
                                   float* col_amax, const nvfp4_outputs* out, void* workspace,
                                   size_t workspace_bytes, cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups, /*k128=*/true);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
@@ -689,7 +686,7 @@ nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int64_t capacity
                                             float* row_amax, float* col_amax, const nvfp4_outputs* out,
                                             void* workspace, size_t workspace_bytes,
                                             int32_t* status_dev, cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups, /*k128=*/true);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_outputs(out, capacity_rows, K, num_groups, do_row, do_col);
@@ -720,7 +717,7 @@ nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int
                                           const int64_t* m_splits_host, int32_t num_groups,
                                           float* row_amax, float* col_amax, const nvfp4_outputs* out,
                                           cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups, /*k128=*/true);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
@@ -783,7 +780,7 @@ nvfp4_status nvfp4_row_post_scale(const float* gemm_out, int64_t rows, int64_t c
 
 nvfp4_status nvfp4_mx_group_cast(const void* x_bf16, int64_t sum_M, int64_t K, const int64_t* m_splits_host,
                                  int32_t num_groups, const nvfp4_mx_outputs* out, cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups, /*k128=*/true);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_mx_outputs(out, sum_M, K, do_row, do_col);
@@ -799,7 +796,7 @@ nvfp4_status nvfp4_mx_group_cast_graphsafe(const void* x_bf16, int64_t capacity_
                                            const int64_t* first_dims_dev, const int64_t* tensor_offsets_dev,
                                            int32_t num_groups, const nvfp4_mx_outputs* out, int32_t* status_dev,
                                            cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups, /*k128=*/true);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_mx_outputs(out, capacity_rows, K, do_row, do_col);

@@ -23,6 +23,21 @@
 
 namespace nvfp4rs {
 
+// ---------------------------------------------- programmatic dependent launch
+//
+// The cast is launched with programmatic stream serialization: its CTAs may
+// start while the kernel before it on the stream (normally the grouped amax)
+// is still finishing. grid_dependency_wait() blocks until that kernel has
+// completed and its writes are visible; a kernel calls it before its first
+// read of anything an earlier kernel may write (x, the amax vectors, device
+// routing). Without a programmatic launch it returns at once.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the kernel after this one on the stream (if launched programmatically)
+// be scheduled now; its own grid_dependency_wait() still waits for this
+// kernel to complete.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 constexpr int kRows = 128;     // rows per tile
 constexpr int kBlockRows = 16; // group sizes are multiples of it: a 16-row block lies in one group
 
@@ -32,13 +47,16 @@ struct RoutingSmem {
   int32_t* off;  // first row of group g; off[E] = routed total
   int32_t E;
   int32_t total;
-  int32_t ok;  // 1 when the routing is usable
+  int32_t ok;      // 1 when the routing is usable
+  int32_t all128;  // 1 when every group is a multiple of 128 rows
 };
 
 // Host split sizes turned into row offsets by the host, passed by value.
 struct HostRouting {
+  static constexpr bool kOnDevice = false;  // the routing is in the kernel parameters
   int32_t E;
   int32_t total;
+  int32_t all128;  // every group a multiple of 128 rows (found by the host)
   int32_t off[NVFP4_MAX_GROUPS + 1];
 
   __device__ __forceinline__ void load(RoutingSmem& s, int32_t* off_smem) const {
@@ -48,6 +66,7 @@ struct HostRouting {
       s.E = E;
       s.total = total;
       s.ok = 1;
+      s.all128 = all128;
     }
     __syncthreads();
   }
@@ -61,11 +80,8 @@ struct HostRouting {
 // With uniform_rows >= 0 the two arrays are absent and every group has
 // uniform_rows rows (the host checked E * uniform_rows <= capacity_rows).
 // Groups whose size is not a multiple of `align` are NVFP4_ERR_UNSUPPORTED.
-// `only_128`: +1 runs the kernel only when every group is a multiple of 128
-// rows, -1 only when some group is not, 0 always; a kernel that does not run
-// returns at once without touching the status (two instantiations of one
-// step are enqueued back to back and exactly one of them runs).
 struct DeviceRouting {
+  static constexpr bool kOnDevice = true;  // the routing is in device memory
   const int64_t* first_dims;
   const int64_t* tensor_offsets;
   int32_t* status;
@@ -74,7 +90,6 @@ struct DeviceRouting {
   int32_t E;
   int32_t align;
   int64_t uniform_rows;
-  int32_t only_128;
 
   __device__ __forceinline__ void load(RoutingSmem& s, int32_t* off_smem) const {
     if (uniform_rows >= 0) {
@@ -84,6 +99,7 @@ struct DeviceRouting {
         s.E = E;
         s.ok = 1;
         s.total = static_cast<int32_t>(E * uniform_rows);
+        s.all128 = uniform_rows % kRows == 0;
       }
       __syncthreads();
       return;
@@ -109,10 +125,10 @@ struct DeviceRouting {
     not_128 = __syncthreads_or(not_128);
     if (threadIdx.x == 0) {
       const int code = bad_routing ? NVFP4_ERR_ROUTING : (bad_align ? NVFP4_ERR_UNSUPPORTED : 0);
-      const bool skip = (only_128 > 0 && not_128) || (only_128 < 0 && !not_128);
       s.off = off_smem;
       s.E = E;
-      s.ok = code == 0 && !skip;
+      s.ok = code == 0;
+      s.all128 = !not_128;
       s.total = code == 0 ? off_smem[E] : 0;
       if (code != 0) gstore(status, static_cast<int32_t>(code));
     }

@@ -69,7 +69,6 @@ def amax(L, x, sum_M, K, splits, row=FAKE, col=FAKE):
 
 @pytest.mark.parametrize("sum_M,K,splits,want", [
     (256, 24, [256], abi.NVFP4_ERR_INVALID_ARG),       # K % 16
-    (256, 144, [256], abi.NVFP4_ERR_UNSUPPORTED),      # K % 128 (fast path)
     (256, 128, [128, 64], abi.NVFP4_ERR_INVALID_ARG),  # splits do not add up
     (256, 128, [384, -128], abi.NVFP4_ERR_INVALID_ARG),  # negative split
     (192, 128, [56, 136], abi.NVFP4_ERR_UNSUPPORTED),  # group not a multiple of 16
@@ -207,3 +206,21 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(abi, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         abi.lib()
+
+
+def test_k_multiple_of_128_only_where_needed(L):
+    """The two-step calls take any K % 16 == 0; the one-launch, MXFP4 and
+    tiled-scale paths need K % 128 == 0 and refuse other K up front."""
+    arr = (ctypes.c_int64 * 1)(256)
+    o = abi.Outputs(row_data=0x10000, row_scale=0x10000, row_s2=0x10000,
+                    col_data=0x10000, col_scale=0x10000, col_s2=0x10000)
+    ws = abi.nvfp4_group_quantize_workspace_bytes(0, 1)
+    assert L.nvfp4_group_quantize(FAKE, 256, 144, arr, 1, FAKE, FAKE, ctypes.byref(o), FAKE, ws, None) == \
+        abi.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_group_quantize_noalloc(FAKE, 256, 144, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_UNSUPPORTED
+    o.scale_layout = abi.NVFP4_SCALE_TILED_128X4
+    assert L.nvfp4_group_cast(FAKE, 256, 144, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_group_cast_graphsafe(FAKE, 256, 144, FAKE, FAKE, 1, FAKE, FAKE, ctypes.byref(o), FAKE,
+                                        None) == abi.NVFP4_ERR_UNSUPPORTED

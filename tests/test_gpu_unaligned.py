@@ -1,24 +1,26 @@
-"""Groups whose sizes are multiples of 16 rows but not of 128, and uniform
-groups, on the GPU (the robustness the TransformerEngine #3649 review asks
-for: supported shapes beyond the 128-row-aligned grouped fast path, and
-uniform expert sizes).
+"""Groups whose sizes are multiples of 16 rows but not of 128, K that is a
+multiple of 16 but not of 128, and uniform groups, on the GPU (the
+robustness the TransformerEngine #3649 review asks for: supported shapes
+beyond the 128-row-aligned grouped fast path, and uniform expert sizes).
 
 Group sizes only need to be multiples of 16 (the colwise block height), so a
 16-row block always lies in one group; a 128-row tile may hold rows of
-several groups, and the last tile may be short. Checked byte for byte
-against the oracle, host-split and graph-safe (which must also agree with
-each other), in both directions and in each alone; uniform graph-safe
-routing (no first_dims / tensor_offsets); the one-launch call, which keeps
-128-row groups, refuses them.
+several groups, and the last tile may be short. K only needs to be a
+multiple of 16 (the rowwise block width); the last 128-column tile may then
+be partial. Checked byte for byte against the oracle, host-split and
+graph-safe (which must also agree with each other, and leave every byte past
+the routed rows untouched), in both directions and in each alone; uniform
+graph-safe routing (no first_dims / tensor_offsets); the one-launch call,
+which keeps 128-row groups and K % 128 == 0, refuses the rest.
 """
 import numpy as np
 import pytest
 import torch
 
-import oracle
 from nvfp4_row_scaled_b200 import abi, workloads
 
-from .helpers import KEYS, assert_identical, gpu_cast, oracle_cast, special_values_case
+from .helpers import KEYS, assert_identical, check_groups_against_oracle, gpu_cast, oracle_cast, \
+    special_values_case
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +53,39 @@ def test_unaligned_against_oracle(K, splits, dist, seed):
     w = workloads.random_case(seed, K, splits, dist=dist)
     assert_identical(gpu_cast(w.x, splits), oracle_cast(w.x, splits), keys=ALL,
                      what=f"K={K} {splits}")
+
+
+KCASES = [
+    (16, [128, 16], "normal", 80),       # K below one TMA box: one 16-column tile
+    (48, [32, 0, 96], "wide", 81),       # second TMA box wholly past K
+    (144, [256], "normal", 82),          # one full and one 16-column tile per row tile
+    (528, [48, 208, 16], "wide", 83),    # K = 4*128 + 16 with unaligned groups
+    (2064, [384, 128], "heavy", 84),     # 128-aligned groups, partial last column tile
+    (7184, [0, 256, 112], "wide", 85),   # DeepSeek-V3 hidden size + 16
+]
+
+
+@pytest.mark.parametrize("K,splits,dist,seed", KCASES)
+def test_k_not_multiple_of_128_against_oracle(K, splits, dist, seed):
+    w = workloads.random_case(seed, K, splits, dist=dist)
+    assert_identical(gpu_cast(w.x, splits), oracle_cast(w.x, splits), keys=ALL,
+                     what=f"K={K} {splits}")
+
+
+@pytest.mark.parametrize("rows,cols", [(True, False), (False, True)])
+def test_k_not_multiple_of_128_single_direction(rows, cols):
+    splits = [48, 0, 208, 16]
+    w = workloads.random_case(86, 400, splits, dist="wide")
+    got = gpu_cast(w.x, splits, rows=rows, cols=cols)
+    want = oracle_cast(w.x, splits, rows=rows, cols=cols)
+    assert set(got) == set(want)
+    assert_identical(got, want)
+
+
+def test_k_not_multiple_of_128_special_values():
+    x, _ = special_values_case(K=400)
+    splits = [48, 0, 80, 16, 112]
+    assert_identical(gpu_cast(x, splits), oracle_cast(x, splits), keys=ALL, what="special values K=400")
 
 
 @pytest.mark.parametrize("rows,cols", [(True, False), (False, True)])
@@ -116,6 +151,40 @@ def test_graphsafe_unaligned_matches_host_split_and_leaves_tail():
         assert np.all(full[k][c:].view(np.uint8) == SENTINEL), k
 
 
+def test_graphsafe_k_not_multiple_of_128_matches_host_split_and_leaves_tail():
+    K, cap = 656, 512
+    splits = [16, 0, 208, 112]  # 336 routed rows of 512
+    w = workloads.random_case(87, K, splits, capacity=cap, dist="wide")
+    x = w.x.cuda()
+    fd, offs = abi.routing_tensors(splits, K)
+    full, st = graphsafe(x, len(splits), fd, offs)
+    assert st == 0
+    total = sum(splits)
+    got = cut(full, total, K)
+    assert_identical(got, gpu_cast(w.x[:total], splits), keys=ALL, what="vs host-split")
+    assert_identical(got, oracle_cast(w.x[:total], splits), keys=ALL, what="vs oracle")
+    for k, c in (("row_data", total), ("row_scale", total), ("row_s2", total), ("row_amax", total),
+                 ("col_data", total * K // 2), ("col_scale", total * K // 16)):
+        assert np.all(full[k][c:].view(np.uint8) == SENTINEL), k
+
+
+def test_k_not_multiple_of_128_refused_by_one_launch_mxfp4_and_tiled():
+    K = 144
+    splits = [128, 128]
+    x = torch.zeros(256, K, dtype=torch.bfloat16, device="cuda")
+    ra, ca = abi.alloc_amax(256, K, 2)
+    out = abi.alloc_outputs(256, K, 2)
+    with pytest.raises(abi.NVFP4Error) as e:
+        abi.nvfp4_group_quantize(x, splits, ra, ca, out, abi.alloc_workspace(0, 2))
+    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
+    with pytest.raises(abi.NVFP4Error) as e:
+        abi.nvfp4_mx_group_cast(x, splits, abi.alloc_mx_outputs(256, K))
+    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
+    with pytest.raises(abi.NVFP4Error) as e:
+        abi.nvfp4_group_cast(x, splits, ra, ca, out, scale_layout=abi.NVFP4_SCALE_TILED_128X4)
+    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("E,m", [(4, 128), (10, 48)])
 def test_graphsafe_uniform_groups(E, m):
     K = 256
@@ -165,23 +234,11 @@ def test_one_launch_refuses_unaligned_groups():
 
 
 @pytest.mark.slow
-def test_deepseek_shape_padded_to_16_full_size_sampled():
-    """Full DeepSeek-V3 routing (8192 tokens) padded to 16 rows: the largest,
-    a middle and a small group against the oracle, every byte."""
+def test_deepseek_shape_padded_to_16_full_size():
+    """Full DeepSeek-V3 routing (8192 tokens) padded to 16 rows, in the
+    benchmark's launch configuration: every byte of every group against the
+    oracle (run group by group over the host's cores)."""
     w = workloads.config3(align=16)
-    got = gpu_cast(w.x, w.m_splits)
-    xb = workloads.bits(w.x)
-    K = w.K
-    offs = workloads.row_offsets(w.m_splits)
-    live = sorted((m, g) for g, m in enumerate(w.m_splits) if m > 0)
-    for _, g in (live[-1], live[len(live) // 2], live[0]):
-        o, m = offs[g], w.m_splits[g]
-        ra, ca = oracle.group_amax(xb[o:o + m], [m])
-        want = oracle.group_cast(xb[o:o + m], [m], ra, ca)
-        np.testing.assert_array_equal(got["row_amax"][o:o + m], ra)
-        np.testing.assert_array_equal(got["col_amax"][g * K:(g + 1) * K], ca)
-        np.testing.assert_array_equal(got["row_data"][o:o + m], want["row_data"])
-        np.testing.assert_array_equal(got["row_scale"][o:o + m], want["row_scale"])
-        np.testing.assert_array_equal(got["col_data"][K * o // 2:K * (o + m) // 2], want["col_data"])
-        np.testing.assert_array_equal(got["col_scale"][K * o // 16:K * (o + m) // 16], want["col_scale"])
-        assert got["col_s2"][g * K:(g + 1) * K].tobytes() == want["col_s2"].tobytes()
+    assert any(m % 128 for m in w.m_splits)
+    check_groups_against_oracle(gpu_cast(w.x, w.m_splits), workloads.bits(w.x), w.m_splits, w.K,
+                                what="deepseek-v3 padded to 16")
