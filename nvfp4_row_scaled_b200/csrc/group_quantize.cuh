@@ -57,8 +57,8 @@
 // the phase complete (acquire), fences (acq_rel, GPU scope) and adds one to
 // the group's done counter (one fence for all the items a sweep finds). The producer waits for a group with acquire
 // loads of that counter, then a proxy fence orders the TMA unit's reads of
-// the maxima after them. adone has two slots per compute group, and a slot
-// is reused only after the publisher acknowledged its previous use (aack), so
+// the maxima after them. adone has kPubSlots slots per compute group, and a
+// slot is reused only after the publisher acknowledged its previous use (aack), so
 // no phase of it can be missed.
 //
 // Workspace (32-bit words, zeroed by the host before the launch):
@@ -186,6 +186,9 @@ constexpr int kControlRegs = 32;
 static_assert(kQGroups * kCastThreads * kComputeRegs + 128 * kControlRegs <= 65536,
               "register split above the launch total");
 constexpr int kQInfo = 4;  // item info ring (item k: entry k % 4)
+// A items a group may have handed to the publisher and not had acknowledged:
+// enough that a run of amax items never waits for the publisher's fence
+constexpr int kPubSlots = 8;
 
 // One compute group's part of shared memory. Item k uses ring entries k % 2
 // (stage, amax copies, encode scales, staged block scales) and k % 4 (info).
@@ -198,11 +201,11 @@ struct alignas(16) QuantGroup {
   uint8_t row_scale[2][8 * kRows];  // B item: staged rowwise block scales
   int32_t item[kQInfo];             // written by the producer before the stage's last arrival
   int32_t grp[kQInfo];
-  int32_t pub_grp[4];               // group of the group's A item a (entry a % 4), for the publisher
+  int32_t pub_grp[kPubSlots];       // group of the group's A item a (entry a % kPubSlots), for the publisher
   uint64_t full[kStages];           // 2 producer arrivals + the tile bytes (+ the amax bytes)
   uint64_t empty[kStages];          // 1 arrival: the group holds the stage's tile in registers
-  uint64_t adone[2];                // 128 arrivals: the group's atomics of an A item are issued
-  uint64_t aack[2];                 // 1 arrival: the publisher has published that A item
+  uint64_t adone[kPubSlots];        // 128 arrivals: the group's atomics of an A item are issued
+  uint64_t aack[kPubSlots];         // 1 arrival: the publisher has published that A item
   int32_t fail;
   int32_t a_final;                  // the group's number of A items once it is finished, else -1
 };
@@ -318,7 +321,7 @@ __device__ __forceinline__ void quantize_publisher(QuantSmem& sm, uint32_t* ws) 
     bool any = false, all = true;
     for (int j = 0; j < kQGroups; j++) {
       const int a = a_pub[j];
-      ready[j] = mbar_test(&sm.grp[j].adone[a & 1], (a >> 1) & 1);
+      ready[j] = mbar_test(&sm.grp[j].adone[a % kPubSlots], (a / kPubSlots) & 1);
       any |= ready[j];
     }
     if (any) {
@@ -327,10 +330,10 @@ __device__ __forceinline__ void quantize_publisher(QuantSmem& sm, uint32_t* ws) 
         if (!ready[j]) continue;
         QuantGroup& pg = sm.grp[j];
         const int a = a_pub[j];
-        const int g = reinterpret_cast<volatile int32_t*>(pg.pub_grp)[a & 3];
+        const int g = reinterpret_cast<volatile int32_t*>(pg.pub_grp)[a % kPubSlots];
         if (NVFP4_STORE_OK(&done[g], 4))
           asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(&done[g]) : "memory");
-        mbar_arrive(&pg.aack[a & 1]);
+        mbar_arrive(&pg.aack[a % kPubSlots]);
         a_pub[j] = a + 1;
       }
     }
@@ -393,7 +396,7 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
         mbar_init(&pg.full[s], 2);
         mbar_init(&pg.empty[s], 1);
       }
-      for (int s = 0; s < 2; s++) {
+      for (int s = 0; s < kPubSlots; s++) {
         mbar_init(&pg.adone[s], kCastThreads);
         mbar_init(&pg.aack[s], 1);
       }
@@ -561,16 +564,17 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
         red_max_u32(dst, S1 << 16);
         red_max_u32(dst + 1, S1 & 0xFFFF0000u);
       }
-      // hand the item to the publisher (slot a % 2, free once A item a - 2 is acknowledged)
+      // hand the item to the publisher (slot a % kPubSlots, free once A item
+      // a - kPubSlots is acknowledged)
       const int a = a_count;
       if (gt == 0) {
-        if (a >= 2 && !mbar_wait(&pg.aack[a & 1], ((a >> 1) - 1) & 1)) {
+        if (a >= kPubSlots && !mbar_wait(&pg.aack[a % kPubSlots], ((a / kPubSlots) - 1) & 1)) {
           pg.fail = 1;  // seen by the group at its next barrier
           raise_abort(abort_word);
         }
-        reinterpret_cast<volatile int32_t*>(pg.pub_grp)[a & 3] = g;
+        reinterpret_cast<volatile int32_t*>(pg.pub_grp)[a % kPubSlots] = g;
       }
-      mbar_arrive(&pg.adone[a & 1]);
+      mbar_arrive(&pg.adone[a % kPubSlots]);
       a_count = a + 1;
     }
   }
