@@ -67,10 +67,24 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources each kernel's code comes from (headers it includes and the file
+# that launches it); a DRAM-traffic record is used only while they hash to the
+# value it was taken on.
+KERNEL_SOURCES = {
+    "group_amax_kernel": ["bounds.cuh", "codec.cuh", "routing.cuh", "group_amax.cuh", "nvfp4rs.cu"],
+    "group_cast_plain_kernel": ["bounds.cuh", "codec.cuh", "routing.cuh", "group_cast.cuh",
+                                "group_cast_plain.cuh", "nvfp4rs.cu"],
+    "group_quantize_kernel": ["bounds.cuh", "codec.cuh", "routing.cuh", "group_cast.cuh", "group_cast_plain.cuh",
+                              "group_amax.cuh", "group_quantize.cuh", "nvfp4rs.cu"],
+}
+
+
+def kernel_source_hash(kernel: str = None) -> str:
+    """Hash of a kernel's sources (all of csrc when the kernel is not listed)."""
     d = os.path.join(ROOT, "nvfp4_row_scaled_b200", "csrc")
+    files = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(d))
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -78,7 +92,7 @@ def kernel_source_hash() -> str:
 
 def traffic_record(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, only if it was
-    taken on the current kernel sources and the same workload."""
+    taken on the current sources of that kernel and the same workload."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
@@ -86,7 +100,7 @@ def traffic_record(kernel: str, workload: str):
     except Exception:
         return None
     r = rec.get(kernel)
-    if not r or r.get("source_hash") != kernel_source_hash() or r.get("workload") != workload:
+    if not r or r.get("source_hash") != kernel_source_hash(kernel) or r.get("workload") != workload:
         return None
     return r.get("bytes_per_launch")
 
@@ -261,7 +275,9 @@ def cpu_baseline(w):
 def other_configs(dev, steps: int):
     """Amax + cast throughput on the other synthetic configurations, beside
     the headline: the tiny and the 8-expert cases (inputs smaller than L2, so
-    L2 is flushed by writing 256 MB before each timed step), the graph-safe
+    L2 is flushed before each timed step: 256 MB are written, then another
+    256 MB read, so that the written lines are back in DRAM before the step
+    starts instead of being written back inside it), the graph-safe
     case (the two graph-safe calls captured once in a CUDA graph and replayed
     over its ten device routings), and the dense single-group case. Each
     figure is the median of per-step CUDA-event times on the launching
@@ -273,6 +289,7 @@ def other_configs(dev, steps: int):
     peak, _ = hbm_peak()
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    clean = torch.zeros(64 * 1024 * 1024, dtype=torch.int32, device=dev)
     n = max(steps, 10)
 
     def median_ms(fn, flush_l2, before=None, reps=n):
@@ -282,6 +299,7 @@ def other_configs(dev, steps: int):
                 before(i)
             if flush_l2:
                 flush.zero_()
+                clean.max()  # reads 256 MB: the flush's dirty lines leave L2 now
             a0 = torch.cuda.Event(enable_timing=True)
             a1 = torch.cuda.Event(enable_timing=True)
             a0.record(stream)
@@ -291,12 +309,15 @@ def other_configs(dev, steps: int):
         torch.cuda.synchronize(dev)
         return statistics.median(a.elapsed_time(b) for a, b in evs)
 
-    def line(w, rows, ms, how):
-        b = algorithmic_bytes(rows, w.K, w.E)["step"]
+    def line(w, rows, ms, how, one_read=False):
+        # algorithmic bytes: two reads of x for the amax + cast pair, one for
+        # the one-launch call (its cast reads x back from L2 where it can)
+        b = algorithmic_bytes(rows, w.K, w.E)["cast" if one_read else "step"]
         return {"workload": w.name, "sum_M": rows, "K": w.K, "experts": w.E, "ms_per_step": round(ms, 4),
                 "value": round(rows * w.K / (ms * 1e-3) / 1e9, 3), "unit": "Gelem/s",
                 "hbm_gbs": round(b / (ms * 1e-3) / 1e9, 1),
-                "hbm_frac_of_peak": round(b / (ms * 1e-3) / 1e9 / peak, 4), "timing": how}
+                "hbm_frac_of_peak": round(b / (ms * 1e-3) / 1e9 / peak, 4),
+                "algorithmic_bytes": "x read once" if one_read else "x read twice (amax, cast)", "timing": how}
 
     res = {}
     for cid in (1, 2, 5):
@@ -313,9 +334,21 @@ def other_configs(dev, steps: int):
         for _ in range(3):
             step()
         small = 2 * R * K < 128 * 1024 * 1024
+        how = "L2 flushed before each step (256 MB written, then 256 MB read)" if small else "input larger than L2"
         ms = median_ms(step, small)
-        res[f"config{cid}"] = line(w, R, ms, "host split; " + ("L2 flushed before each step" if small
-                                                               else "input larger than L2"))
+        res[f"config{cid}"] = line(w, R, ms, "host split; " + how)
+        if all(m % 128 == 0 for m in w.m_splits) and K % 128 == 0:  # the one-launch call's shapes
+            ws = abi.alloc_workspace(0, E, dev)
+
+            def one():
+                abi.nvfp4_group_quantize(x, w.m_splits, ra, ca, out, ws)
+
+            for _ in range(3):
+                one()
+            ms1 = median_ms(one, small)
+            res[f"config{cid}_one_launch"] = line(w, R, ms1, "nvfp4_group_quantize (one launch), host split; " + how,
+                                                  one_read=True)
+            del ws
         del x, ra, ca, out
 
     # graph-safe: routing only in device first_dims / tensor_offsets
@@ -352,6 +385,29 @@ def other_configs(dev, steps: int):
     res["config4"] = line(w, cap, ms, "CUDA-graph replay, routing rewritten on the device before each "
                                       "replay (ten routings, twice); input larger than L2")
 
+    # the one-launch graph-safe call, captured and replayed the same way
+    ws = abi.alloc_workspace(cap, E, dev)
+
+    def gs_one():
+        abi.nvfp4_group_quantize_graphsafe(x, fd, offs, ra, ca, out, ws, status)
+
+    set_routing(0)
+    gs_one()
+    torch.cuda.synchronize(dev)
+    graph1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph1):
+        gs_one()
+    for i in range(3):
+        set_routing(i)
+        graph1.replay()
+    ms = median_ms(graph1.replay, False, before=set_routing, reps=2 * len(routes))
+    if int(status.item()) != 0:
+        raise RuntimeError(f"graph-safe one-launch replay reported status {int(status.item())}")
+    res["config4_one_launch"] = line(w, cap, ms, "nvfp4_group_quantize_graphsafe (one launch) in a CUDA graph, "
+                                                 "replayed over the ten routings twice; input larger than L2",
+                                     one_read=True)
+    del graph1, ws
+
     def hs_step():
         abi.nvfp4_group_amax(x, w.routings[0], ra, ca)
         abi.nvfp4_group_cast(x, w.routings[0], ra, ca, out)
@@ -361,7 +417,7 @@ def other_configs(dev, steps: int):
     ms = median_ms(hs_step, False)
     res["config4_host_split"] = line(w, cap, ms, "the same input and its first routing through the host-split "
                                                  "calls; input larger than L2")
-    del graph, x, ra, ca, out, flush
+    del graph, x, ra, ca, out, flush, clean
     return res
 
 

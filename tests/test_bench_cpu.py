@@ -35,19 +35,30 @@ def _fake_root(tmp_path, record):
     (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(record))
 
 
+def test_kernel_source_lists_exist():
+    d = os.path.join(ROOT, "nvfp4_row_scaled_b200", "csrc")
+    for files in bench.KERNEL_SOURCES.values():
+        for f in files:
+            assert os.path.exists(os.path.join(d, f)), f
+
+
 def test_traffic_record_only_for_the_sources_it_was_measured_on(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     _fake_root(tmp_path, {})
-    h = bench.kernel_source_hash()
+    h = bench.kernel_source_hash("group_cast_plain_kernel")
     rec = {"group_cast_plain_kernel": {"workload": "w", "source_hash": h, "bytes_per_launch": 123}}
     (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
     assert bench.traffic_record("group_cast_plain_kernel", "w") == 123
     assert bench.traffic_record("group_cast_plain_kernel", "other workload") is None
     assert bench.traffic_record("group_amax_kernel", "w") is None
-    # any change to a kernel source retires the record
+    # a change to a source of another kernel only keeps the record
+    f = tmp_path / "nvfp4_row_scaled_b200" / "csrc" / "mx_cast.cuh"
+    f.write_text(f.read_text() + "\n")
+    assert bench.traffic_record("group_cast_plain_kernel", "w") == 123
+    # any change to one of the kernel's own sources retires it
     f = tmp_path / "nvfp4_row_scaled_b200" / "csrc" / "codec.cuh"
     f.write_text(f.read_text() + "\n")
-    assert bench.kernel_source_hash() != h
+    assert bench.kernel_source_hash("group_cast_plain_kernel") != h
     assert bench.traffic_record("group_cast_plain_kernel", "w") is None
 
 
