@@ -55,9 +55,10 @@
  *    NVFP4_ERR_INVALID_ARG). Else NVFP4_ERR_UNSUPPORTED: every group size
  *    m_g % 16 == 0 (the colwise block height), num_groups <=
  *    NVFP4_MAX_GROUPS, rows < 2^31, and every pointer 16-byte aligned. The
- *    one-launch calls, the MXFP4 calls and the 128x4-tiled scale layout also
- *    need K % 128 == 0 and m_g % 128 == 0 (the 128-row alignment of the
- *    grouped GEMM's scale layout). 128-row tiles inside one group on the
+ *    one-launch calls and the 128x4-tiled scale layout also need
+ *    K % 128 == 0 and m_g % 128 == 0 (the 128-row alignment of the grouped
+ *    GEMM's scale layout); the MXFP4 calls need K % 32 == 0 (else
+ *    NVFP4_ERR_INVALID_ARG) and m_g % 32 == 0 (their block size). 128-row tiles inside one group on the
  *    128-row grid, with K % 128 == 0, take the fastest path; the rest is
  *    handled at the tile's edges in the same kernel (a 128-row tile may then
  *    hold rows of several groups, the last row tile may be short, and the
@@ -322,9 +323,9 @@ NVFP4RS_API nvfp4_status nvfp4_dequantize(const uint8_t* data, const uint8_t* sc
  *   s = clamp(floor(log2 a) - 2, -127, 127)   (a == 0 gives -127)
  *   scale byte = s + 127;  code_j = E2M1_rne_satfinite(x_j * 2^-s), sign kept
  *   dequantize: x_hat = e2m1(code) * 2^(scale - 127)
- * Same grouped structure as the NVFP4 cast; groups must be multiples of 128
- * rows and K % 128 == 0 (else NVFP4_ERR_UNSUPPORTED). One read of x, one
- * launch: no amax step. */
+ * Same grouped structure and kernel organisation as the NVFP4 cast; groups
+ * must be multiples of 32 rows (else NVFP4_ERR_UNSUPPORTED) and K a multiple
+ * of 32 (else NVFP4_ERR_INVALID_ARG). One read of x, one launch: no amax step. */
 typedef struct {
   uint8_t* row_data;  /* [rows, K/2]                               */
   uint8_t* row_scale; /* [rows, K/32] E8M0                         */
@@ -338,8 +339,9 @@ NVFP4RS_API nvfp4_status nvfp4_mx_group_cast(const void* x_bf16, int64_t sum_M, 
                                  const nvfp4_mx_outputs* out, cudaStream_t stream);
 
 /* Grouped MXFP4 cast, graph-safe routing (arguments and status as
- * nvfp4_group_cast_graphsafe; a group that is not a multiple of 128 rows is
- * NVFP4_ERR_UNSUPPORTED on the device). Byte-identical to the host-split call. */
+ * nvfp4_group_cast_graphsafe; a group that is not a multiple of 32 rows is
+ * NVFP4_ERR_UNSUPPORTED on the device). Byte-identical to the host-split call;
+ * one launch whatever the device routing holds. */
 NVFP4RS_API nvfp4_status nvfp4_mx_group_cast_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
                                            const int64_t* first_dims_dev,
                                            const int64_t* tensor_offsets_dev, int32_t num_groups,

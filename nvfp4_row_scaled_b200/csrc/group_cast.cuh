@@ -47,22 +47,6 @@ struct CastOut {
   int32_t tiled_scales;  // nonzero: both scale outputs in the 128x4-tiled layout
 };
 
-// Output staging of one tile.
-struct CastStage {
-  uint8_t col_data[kCols * 64];  // [column][64 B]; 8-byte slot b at (b ^ (column/8 % 8))
-  uint8_t col_scale[8 * kCols];  // [row block][column]
-  uint8_t row_scale[8 * kRows];  // [column block][row]
-};
-
-// Dynamic shared memory of the MXFP4 cast kernel; `off` (E+1 int32) follows it.
-struct CastSmem {
-  uint8_t tile[kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
-  uint64_t full[kStages];
-};
-
-constexpr size_t cast_smem_bytes(int E) {
-  return ((sizeof(CastSmem) + 15) & ~size_t{15}) + sizeof(int32_t) * (E + 1);
-}
 
 // ------------------------------------------------------------- TMA / mbarrier
 
@@ -137,15 +121,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// Load the 128 x 128 tile (row tile rt, column tile ct) into stage s. Both
-// boxes start at a column that is a multiple of 64 (128 bytes).
-__device__ __forceinline__ void issue_tile_at(CastSmem& sm, const CUtensorMap* map, int s, int rt,
-                                              int ct, uint64_t policy) {
-  mbar_expect_tx(&sm.full[s], kTileBytes);
-  tma_load_2d(sm.tile[s], map, ct * kCols, rt * kRows, &sm.full[s], policy);
-  tma_load_2d(sm.tile[s] + kBoxBytes, map, ct * kCols + kBoxCols, rt * kRows, &sm.full[s], policy);
-}
-
 // Untiled bulk copy global -> shared (16-byte aligned, multiple of 16 bytes),
 // completion counted on `bar`. No multicast.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -157,15 +132,8 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Tile number `tl` of the row-major tile order (read once: evict first).
-__device__ __forceinline__ void issue_tile(CastSmem& sm, const CUtensorMap* map, int s, int tl,
-                                           int n_ct) {
-  const int rt = tl / n_ct;
-  issue_tile_at(sm, map, s, rt, tl - rt * n_ct, policy_evict_first());
-}
-
-// Lane (cc, h) of warp w: rows rl .. rl+15 (rl = 16 * (2w + h)), columns
-// 8cc .. 8cc+7 of the swizzled 128 x 128 tile at `tile` (two 64-column boxes).
+// A lane's patch: rows rl .. rl+15, columns 8cc .. 8cc+7 of the swizzled
+// 128 x 128 tile at `tile` (two 64-column boxes).
 __device__ __forceinline__ void load_patch(const uint8_t* tile, int cc, int rl, uint4 (&v)[16]) {
   const uint8_t* tb = tile + (cc >> 3) * kBoxBytes + rl * 128;
   const int j = cc & 7;
@@ -238,19 +206,6 @@ __device__ __forceinline__ void encode_codes(const uint4 (&v)[16], const float (
     }
   }
 }
-
-// The staging sink of encode_codes: the column words of lane (cc, rb) go to
-// st.col_data, 8 bytes per column at slot rb ^ (cc % 8).
-struct StageColSink {
-  CastStage& st;
-  int cc, rb;
-  __device__ __forceinline__ void operator()(int half, const uint32_t (&cw)[8]) const {
-    const int slot = rb ^ (cc & 7);
-#pragma unroll
-    for (int q = 0; q < 8; q++)
-      *reinterpret_cast<uint32_t*>(&st.col_data[(8 * cc + q) * 64 + 8 * slot + 4 * half]) = cw[q];
-  }
-};
 
 // The shared tables a tile's encode reads: the E4M3 table of the block-scale
 // shortcut, and S_enc of the tile's 128 rows.
@@ -371,24 +326,6 @@ __device__ __forceinline__ uint2 tiled_piece(const uint8_t* stg, int t) {
             (static_cast<uint32_t>(stg[2 * kRows + r]) << 16) | (static_cast<uint32_t>(stg[3 * kRows + r]) << 24);
   }
   return make_uint2(w[0], w[1]);
-}
-
-// The staged colwise codes of a whole tile of a 128-aligned group: 64 bytes
-// per column (four 16-byte pieces) into the group's transposed slice.
-__device__ __forceinline__ void store_col_data(const CastStage& st, uint8_t* col_data, int K, int32_t o_g,
-                                               int64_t m_g, int32_t r0, int c0, int t, uint64_t keep) {
-  const size_t half_m = static_cast<size_t>(m_g) >> 1;
-  uint8_t* gd = col_data + (static_cast<size_t>(K) * o_g >> 1) + ((r0 - o_g) >> 1);
-#pragma unroll
-  for (int kk = 0; kk < 4; kk++) {
-    const int u = kk * kCastThreads + t;
-    const int col = u >> 2, part = u & 3;
-    const int sw = (col >> 3) & 7;
-    const uint2 lo = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part) ^ sw)]);
-    const uint2 hi = *reinterpret_cast<const uint2*>(&st.col_data[col * 64 + 8 * ((2 * part + 1) ^ sw)]);
-    st_global_u4_hint(gd + static_cast<size_t>(c0 + col) * half_m + 16 * part, make_uint4(lo.x, lo.y, hi.x, hi.y),
-                      keep);
-  }
 }
 
 // The staged block scales of a tile of a 128-aligned group: colwise

@@ -32,6 +32,7 @@ using namespace nvfp4rs;
 namespace {
 
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - kRows;
+constexpr int kMxBlock = 32;  // MXFP4 block: 32 elements along K (rowwise) and along a group's rows (colwise)
 constexpr int kMaxAmaxCols = 32768;  // columns per amax CTA (dynamic shared memory)
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -477,23 +478,24 @@ nvfp4_status check_mx_outputs(const nvfp4_mx_outputs* out, int64_t rows, int64_t
 template <class Routing>
 nvfp4_status launch_mx_cast(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
                             const nvfp4_mx_outputs* out, cudaStream_t stream) {
-  const int64_t tiles = (rows / kRows) * (K / kCols);
+  const int64_t tiles = ((rows + kRows - 1) / kRows) * ((K + kCols - 1) / kCols);
   if (tiles == 0) return NVFP4_OK;
   CUtensorMap map;
   if (!x_tensor_map(&map, x, rows, K)) return NVFP4_ERR_CUDA;
   auto kernel = mx_cast_kernel<Routing>;
-  const size_t smem = cast_smem_bytes(E) + 1024;
+  const size_t smem = mx_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return NVFP4_ERR_CUDA;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCastThreads, smem) != cudaSuccess)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPThreads, smem) != cudaSuccess)
     return NVFP4_ERR_CUDA;
   if (per_sm < 1) return NVFP4_ERR_UNSUPPORTED;
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
-  if (tiles < grid) grid = tiles;
+  const int64_t units = (tiles + kPGroups - 1) / kPGroups;
+  if (units < grid) grid = units;
   const MxOut o{out->row_data, out->row_scale, out->col_data, out->col_scale};
 #ifdef NVFP4_CHECK_BOUNDS
   {
@@ -510,7 +512,7 @@ nvfp4_status launch_mx_cast(const Routing& routing, const void* x, int64_t rows,
 #endif
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kCastThreads);
+  cfg.blockDim = dim3(kPThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, map, static_cast<int32_t>(K), o));
@@ -780,13 +782,14 @@ nvfp4_status nvfp4_row_post_scale(const float* gemm_out, int64_t rows, int64_t c
 
 nvfp4_status nvfp4_mx_group_cast(const void* x_bf16, int64_t sum_M, int64_t K, const int64_t* m_splits_host,
                                  int32_t num_groups, const nvfp4_mx_outputs* out, cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups, /*k128=*/true);
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
   if (s != NVFP4_OK) return s;
+  if (K % kMxBlock != 0) return NVFP4_ERR_INVALID_ARG;
   bool do_row = false, do_col = false;
   s = check_mx_outputs(out, sum_M, K, do_row, do_col);
   if (s != NVFP4_OK) return s;
   static thread_local HostRouting routing;
-  s = host_routing(m_splits_host, num_groups, sum_M, routing, kRows);
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kMxBlock);  // a 32-row block lies in one group
   if (s != NVFP4_OK) return s;
   if (!do_row && !do_col) return NVFP4_OK;
   return launch_mx_cast(routing, x_bf16, sum_M, K, num_groups, out, stream);
@@ -796,13 +799,14 @@ nvfp4_status nvfp4_mx_group_cast_graphsafe(const void* x_bf16, int64_t capacity_
                                            const int64_t* first_dims_dev, const int64_t* tensor_offsets_dev,
                                            int32_t num_groups, const nvfp4_mx_outputs* out, int32_t* status_dev,
                                            cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups, /*k128=*/true);
+  nvfp4_status s = check_shape(x_bf16, capacity_rows, K, num_groups);
   if (s != NVFP4_OK) return s;
+  if (K % kMxBlock != 0) return NVFP4_ERR_INVALID_ARG;
   bool do_row = false, do_col = false;
   s = check_mx_outputs(out, capacity_rows, K, do_row, do_col);
   if (s != NVFP4_OK) return s;
   DeviceRouting routing;
-  s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups, kRows,
+  s = device_routing(first_dims_dev, tensor_offsets_dev, status_dev, K, capacity_rows, num_groups, kMxBlock,
                      routing);
   if (s != NVFP4_OK) return s;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));

@@ -184,9 +184,11 @@ def test_mx_host_checks(L):
     o = abi.MxOutputs(row_data=0x10000, row_scale=None)  # partial direction
     assert L.nvfp4_mx_group_cast(FAKE, 256, 128, arr, 2, ctypes.byref(o), None) == abi.NVFP4_ERR_INVALID_ARG
     o = abi.MxOutputs(row_data=0x10000, row_scale=0x10000)
-    assert L.nvfp4_mx_group_cast(FAKE, 256, 144, arr, 2, ctypes.byref(o), None) == abi.NVFP4_ERR_UNSUPPORTED
-    arr2 = (ctypes.c_int64 * 2)(64, 192)
-    assert L.nvfp4_mx_group_cast(FAKE, 256, 128, arr2, 2, ctypes.byref(o), None) == abi.NVFP4_ERR_UNSUPPORTED
+    # K must be a multiple of the 32-element block, as in the oracle
+    assert L.nvfp4_mx_group_cast(FAKE, 256, 144, arr, 2, ctypes.byref(o), None) == abi.NVFP4_ERR_INVALID_ARG
+    # groups must be multiples of 32 rows (a colwise block lies in one group)
+    arr2 = (ctypes.c_int64 * 2)(48, 208)
+    assert L.nvfp4_mx_group_cast(FAKE, 256, 160, arr2, 2, ctypes.byref(o), None) == abi.NVFP4_ERR_UNSUPPORTED
     f = L.nvfp4_mx_dequantize
     assert f(FAKE, FAKE, 4, 48, FAKE, None) == abi.NVFP4_ERR_INVALID_ARG  # cols % 32
     assert f(FAKE, FAKE, 4, 64, ctypes.c_void_p(0x10008), None) == abi.NVFP4_ERR_UNSUPPORTED

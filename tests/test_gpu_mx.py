@@ -1,9 +1,10 @@
 """Grouped MXFP4 cast on the GPU (E2M1, blocks of 32, E8M0 scales; the
 "E2M1/block-32/E8M0" configuration of TransformerEngine #3824, Testing),
 byte for byte against the oracle: both directions and each alone, empty
-groups, several widths, special values (zeros, subnormals, ties, values near
-the bf16 maximum), the graph-safe twin (identical, untouched tail, refused
-routing), and the MXFP4 dequantize (bit-exact fp32).
+groups, several widths, groups of any multiple of 32 rows and K any multiple
+of 32, special values (zeros, subnormals, ties, values near the bf16
+maximum), the graph-safe twin (identical, untouched tail, refused routing),
+and the MXFP4 dequantize (bit-exact fp32).
 """
 import numpy as np
 import pytest
@@ -99,19 +100,79 @@ def test_graphsafe_identical_and_tail_untouched():
         assert np.all(v[cut[k]:] == 0xA5), k
 
 
-def test_graphsafe_refuses_unaligned_groups():
+def test_graphsafe_refuses_groups_off_the_32_row_grid():
     K = 256
     x = torch.zeros(256, K, dtype=torch.bfloat16, device="cuda")
-    fd = torch.tensor([64, 192], dtype=torch.int64, device="cuda")
-    offs = torch.tensor([0, 64 * K, 256 * K], dtype=torch.int64, device="cuda")
+    fd = torch.tensor([48, 208], dtype=torch.int64, device="cuda")
+    offs = torch.tensor([0, 48 * K, 256 * K], dtype=torch.int64, device="cuda")
     out = abi.alloc_mx_outputs(256, K)
+    for t in out.values():
+        t.fill_(0xA5)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     abi.nvfp4_mx_group_cast_graphsafe(x, fd, offs, out, st)
     torch.cuda.synchronize()
     assert int(st.item()) == abi.NVFP4_ERR_UNSUPPORTED
+    for k, v in out.items():
+        assert bool(torch.all(v == 0xA5)), k
     with pytest.raises(abi.NVFP4Error) as e:
-        abi.nvfp4_mx_group_cast(x, [64, 192], out)
+        abi.nvfp4_mx_group_cast(x, [48, 208], out)
     assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
+
+
+# groups of any multiple of 32 rows and K any multiple of 32: tiles that a
+# group boundary crosses, groups off the 128-row grid, a short last row tile,
+# a partial last column tile
+UNALIGNED = [
+    (128, [32], "normal", 111),                        # one short tile
+    (256, [96, 0, 32, 160, 64], "wide", 112),          # several groups per tile, empty in the middle
+    (160, [128, 32, 0, 96], "heavy", 113),             # K = 128 + 32
+    (32, [64, 224], "normal", 114),                    # K below one TMA box
+    (1056, [288, 0, 416, 96], "wide", 115),            # K = 8*128 + 32, groups straddling tiles
+    (7168, [224, 0, 32, 96], "wide", 116),
+]
+
+
+@pytest.mark.parametrize("K,splits,dist,seed", UNALIGNED)
+def test_unaligned_groups_and_k(K, splits, dist, seed):
+    w = workloads.random_case(seed, K, splits, dist=dist)
+    check(gpu_mx(w.x, splits), oracle.mx_group_cast(workloads.bits(w.x), splits), f"K={K} {splits}")
+
+
+@pytest.mark.parametrize("rows,cols", [(True, False), (False, True)])
+def test_unaligned_single_direction(rows, cols):
+    splits = [96, 0, 224, 32]
+    w = workloads.random_case(117, 416, splits, dist="wide")
+    check(gpu_mx(w.x, splits, rows, cols), oracle.mx_group_cast(workloads.bits(w.x), splits, rows, cols),
+          f"rows={rows}")
+
+
+def test_unaligned_special_values():
+    x, _ = special_values_case(K=416)
+    splits = [96, 0, 64, 32, 64]
+    check(gpu_mx(x, splits), oracle.mx_group_cast(workloads.bits(x), splits), "special values K=416")
+
+
+def test_graphsafe_unaligned_identical_and_tail_untouched():
+    K, cap = 544, 768
+    splits = [32, 0, 288, 96]  # 416 routed rows of 768
+    w = workloads.random_case(118, K, splits, capacity=cap, dist="wide")
+    x = w.x.cuda()
+    fd, offs = abi.routing_tensors(splits, K)
+    out = abi.alloc_mx_outputs(cap, K)
+    for t in out.values():
+        t.fill_(0xA5)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.nvfp4_mx_group_cast_graphsafe(x, fd, offs, out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    total = sum(splits)
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    cut = {"row_data": total, "row_scale": total, "col_data": total * K // 2, "col_scale": total * K // 32}
+    head = {k: v[:cut[k]] for k, v in got.items()}
+    check(head, gpu_mx(w.x[:total], splits), "graph-safe vs host-split")
+    check(head, oracle.mx_group_cast(workloads.bits(w.x[:total]), splits), "graph-safe vs oracle")
+    for k, v in got.items():
+        assert np.all(v[cut[k]:] == 0xA5), k
 
 
 def test_dequantize_bit_exact():

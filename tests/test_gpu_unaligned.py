@@ -168,7 +168,7 @@ def test_graphsafe_k_not_multiple_of_128_matches_host_split_and_leaves_tail():
         assert np.all(full[k][c:].view(np.uint8) == SENTINEL), k
 
 
-def test_k_not_multiple_of_128_refused_by_one_launch_mxfp4_and_tiled():
+def test_k_not_multiple_of_128_refused_by_one_launch_and_tiled():
     K = 144
     splits = [128, 128]
     x = torch.zeros(256, K, dtype=torch.bfloat16, device="cuda")
@@ -176,9 +176,6 @@ def test_k_not_multiple_of_128_refused_by_one_launch_mxfp4_and_tiled():
     out = abi.alloc_outputs(256, K, 2)
     with pytest.raises(abi.NVFP4Error) as e:
         abi.nvfp4_group_quantize(x, splits, ra, ca, out, abi.alloc_workspace(0, 2))
-    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
-    with pytest.raises(abi.NVFP4Error) as e:
-        abi.nvfp4_mx_group_cast(x, splits, abi.alloc_mx_outputs(256, K))
     assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
     with pytest.raises(abi.NVFP4Error) as e:
         abi.nvfp4_group_cast(x, splits, ra, ca, out, scale_layout=abi.NVFP4_SCALE_TILED_128X4)
