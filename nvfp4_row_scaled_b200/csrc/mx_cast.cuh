@@ -15,7 +15,7 @@
 // below 8 in magnitude).
 //
 // Structure: the NVFP4 cast kernel's (group_cast_plain.cuh) -- one CTA per
-// SM of three warp groups, each with its own two-stage TMA ring, 16-row x
+// SM of three warp groups, each with its own one-stage TMA ring, 16-row x
 // 8-column lane patches, rowwise and colwise codes straight from registers to
 // global memory -- with the MXFP4 block rule and no amax inputs. A rowwise
 // block (32 columns) spans four lanes (lanes ^1, ^2), a colwise block (32
@@ -113,13 +113,13 @@ struct alignas(16) MxGroup {
   uint8_t col_scale[2][4 * kCols];  // staged colwise scales [32-row block][column]
   uint8_t row_scale[2][4 * kRows];  // staged rowwise scales [32-column block][row]
   TileInfo info[kPInfo];
-  uint64_t full[kStages];
+  uint64_t full;  // the stage's mbarrier: tile k completes phase k % 2
   int32_t fail;
 };
 
 // Dynamic shared memory of the kernel; `off` (E+1 int32) follows it.
 struct MxSmem {
-  uint8_t tile[kPGroups][kStages][kTileBytes];  // at offset 0 of a 1024-byte aligned block
+  uint8_t tile[kPGroups][kTileBytes];  // one stage per group, at offset 0 of a 1024-byte aligned block
   MxGroup grp[kPGroups];
   RoutingSmem rs;
 };
@@ -128,9 +128,9 @@ constexpr size_t mx_smem_bytes(int E) {
   return ((sizeof(MxSmem) + 15) & ~size_t{15}) + sizeof(int32_t) * (E + 1);
 }
 
-// One thread of the group: tile (rt, ct) -- the group's k-th -- into stage s
-// with its tile info (as plain_issue, without amax copies).
-__device__ __forceinline__ void mx_issue(MxGroup& pg, uint8_t* stage, const CUtensorMap* map, int s, int k, int rt,
+// One thread of the group: tile (rt, ct) -- the group's k-th -- into the
+// stage with its tile info (as plain_issue, without amax copies).
+__device__ __forceinline__ void mx_issue(MxGroup& pg, uint8_t* stage, const CUtensorMap* map, int k, int rt,
                                          int ct, const RoutingSmem& rs, int K, bool k128) {
   const int32_t r0 = rt * kRows;
   const int c0 = ct * kCols;
@@ -155,10 +155,10 @@ __device__ __forceinline__ void mx_issue(MxGroup& pg, uint8_t* stage, const CUte
       inf.gb[b] = gb;
     }
   }
-  mbar_expect_tx(&pg.full[s], kTileBytes);
+  mbar_expect_tx(&pg.full, kTileBytes);
   const uint64_t pol = policy_evict_first();
-  tma_load_2d(stage, map, c0, r0, &pg.full[s], pol);
-  tma_load_2d(stage + kBoxBytes, map, c0 + kBoxCols, r0, &pg.full[s], pol);
+  tma_load_2d(stage, map, c0, r0, &pg.full, pol);
+  tma_load_2d(stage + kBoxBytes, map, c0 + kBoxCols, r0, &pg.full, pol);
 }
 
 // The staged scales of a tile: a plain tile's as 4 bytes per column and per
@@ -230,27 +230,26 @@ __device__ __forceinline__ void mx_tiles(MxSmem& sm, MxGroup& pg, const Routing&
   bool failed = false;
   int rtp = 0, ctp = 0;
   for (int tl = first; tl < n_tiles; tl += G, k++) {
-    const int s = k & 1;
     const int32_t r0 = rt * kRows;
     const int c0 = ct * kCols;
-    const bool ok = mbar_wait(&pg.full[s], (k >> 1) & 1);
+    const bool ok = mbar_wait(&pg.full, k & 1);
     if (!ok) pg.fail = 1;
     uint4 v[16];
-    load_patch(sm.tile[j][s], cc, rl, v);
+    load_patch(sm.tile[j], cc, rl, v);
     group_bar(bar_id);
     if (pg.fail) {
       failed = true;
       break;
     }
-    // every patch of tile k is in registers: its stage takes tile k+2
-    if (gt == 32 * (k & 3) && tl + 2 * G < n_tiles) {
-      int rt2 = rt + 2 * Gq, ct2 = ct + 2 * Gr;
-      while (ct2 >= n_ct) {
+    // every patch of tile k is in registers: the stage takes tile k+1
+    if (gt == 32 * (k & 3) && tl + G < n_tiles) {
+      int rt2 = rt + Gq, ct2 = ct + Gr;
+      if (ct2 >= n_ct) {
         ct2 -= n_ct;
         rt2++;
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mx_issue(pg, sm.tile[j][s], tmap, s, k + 2, rt2, ct2, rs, K, k128);
+      mx_issue(pg, sm.tile[j], tmap, k + 1, rt2, ct2, rs, K, k128);
     }
     if (k >= 1)  // the previous tile's staged scales (complete since the barrier)
       mx_store_scales<kGeneral>(pg, (k - 1) & 1, pg.info[(k - 1) % kPInfo], out, rs, K, rtp * kRows, ctp * kCols, gt,
@@ -289,8 +288,8 @@ __device__ __forceinline__ void mx_tiles(MxSmem& sm, MxGroup& pg, const Routing&
                               do_row, do_col);
   }
   if (failed && gt == 0) {
-    // drain the loads this group issued and did not consume (tiles k, k+1)
-    for (int jj = k; jj <= k + 1 && first + jj * G < n_tiles; jj++) mbar_wait(&pg.full[jj & 1], (jj >> 1) & 1);
+    // drain the load this group issued and did not consume (tile k)
+    mbar_wait(&pg.full, k & 1);
     routing.report(NVFP4_ERR_TIMEOUT);
   }
 }
@@ -322,23 +321,14 @@ mx_cast_kernel(const __grid_constant__ Routing routing, const __grid_constant__ 
   const int G = gridDim.x * kPGroups;
   const int first = j * gridDim.x + blockIdx.x;  // groups running together take neighbouring tiles
   if (gt == 0) {
-    for (int s = 0; s < kStages; s++) mbar_init(&pg.full[s], 1);
+    mbar_init(&pg.full, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     pg.fail = 0;
   }
   __syncthreads();
   if (gt == 0) {
-    const int Gq = G / n_ct, Gr = G - Gq * n_ct;
-    int rti = first / n_ct, cti = first - rti * n_ct;
-    for (int k = 0; k < kStages && first + k * G < n_tiles; k++) {
-      mx_issue(pg, sm.tile[j][k], &tmap, k, k, rti, cti, rs, K, k128);
-      cti += Gr;
-      rti += Gq;
-      if (cti >= n_ct) {
-        cti -= n_ct;
-        rti++;
-      }
-    }
+    const int rti = first / n_ct, cti = first - rti * n_ct;
+    if (first < n_tiles) mx_issue(pg, sm.tile[j], &tmap, 0, rti, cti, rs, K, k128);
   }
   // every group a multiple of 128 rows and K % 128 == 0: every tile is plain
   if (rs.all128 && k128)

@@ -280,6 +280,7 @@ nvfp4_status launch_cast(const Routing& routing, const void* x, int64_t rows, in
   const bool tiled = out->scale_layout == NVFP4_SCALE_TILED_128X4;
   auto kernel = tiled ? group_cast_plain_kernel<Routing, true> : group_cast_plain_kernel<Routing, false>;
   const int64_t units = (tiles + kPGroups - 1) / kPGroups;
+  static_assert(plain_smem_bytes(NVFP4_MAX_GROUPS) + 1024 <= 227 * 1024, "cast kernel shared memory");
   const size_t smem = plain_smem_bytes(E) + 1024;  // + room to align the block to 1024 bytes
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
