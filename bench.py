@@ -752,7 +752,7 @@ def main():
                       "hbm_frac_of_peak": round(deq_mx_bytes / (deq_mx_ms * 1e-3) / 1e9 / peak, 4)},
         },
         "other_configs": others,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,  # per step: zero_f32_kernel, group_amax_kernel, group_cast_plain_kernel
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)

@@ -31,7 +31,10 @@
 // CTA rank 0, which writes row_amax. Column maxima go to col_amax with one
 // unsigned atomic max per column per CTA (non-negative floats order like
 // their bit patterns, and max is order-free, so the result is deterministic).
-// col_amax must be zero before the launch (the host enqueues a memset).
+// col_amax must be zero before the kernel's first atomic: the host enqueues
+// zero_f32_kernel just before it and launches this kernel programmatically
+// after it, so that the reads of x overlap the zeroing; every atomic on
+// col_amax comes after grid_dependency_wait().
 #pragma once
 
 #include <cooperative_groups.h>
@@ -58,6 +61,15 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 __device__ __forceinline__ void red_max_u32(float* addr, uint32_t v) {
   if (!NVFP4_STORE_OK(addr, 4)) return;
   asm volatile("red.global.max.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+// Zeroes n floats, after letting the kernel launched after it on the stream
+// start at once (that kernel waits for this one before it touches p).
+__global__ void __launch_bounds__(256) zero_f32_kernel(float* __restrict__ p, int64_t n) {
+  launch_dependents();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    gstore(&p[i], 0.0f);
 }
 
 template <class Routing>
@@ -169,6 +181,7 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
       }
       if (mixed) {  // straight to this lane's group (a mixed tile is rare)
         if (lane_ok && col_ok && col_amax != nullptr) {
+          grid_dependency_wait();  // col_amax is zero
           float* dst = col_amax + static_cast<size_t>(g_lane) * K + c_glb;
           const uint32_t w[4] = {c0 & 0x7FFF7FFFu, c1 & 0x7FFF7FFFu, c2 & 0x7FFF7FFFu, c3 & 0x7FFF7FFFu};
 #pragma unroll
@@ -194,6 +207,7 @@ group_amax_kernel(const __grid_constant__ Routing routing, const uint4* __restri
   }
   __syncthreads();
   if (active && !mixed && col_amax != nullptr) {
+    grid_dependency_wait();  // col_amax is zero
     float* dst = col_amax + static_cast<size_t>(g_first) * K;
     for (int c = t; c < cols; c += kAmaxThreads) {
       const int gc = (((c >> 7) * cn + rank) << 7) | (c & 127);

@@ -8,6 +8,7 @@
 // the same kernel templates with a different routing front-end
 // (routing.cuh), which is what makes their outputs byte-identical
 // (TransformerEngine #3649, grouped row-scaled NVFP4 cast, Description).
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -223,11 +224,14 @@ bool x_tensor_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// col_amax (when given) is zeroed here first, by a kernel after which the
+// amax kernel is launched programmatically (group_amax.cuh).
 template <class Routing>
 nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t rows, int64_t K, int32_t E,
                          float* row_amax, float* col_amax, cudaStream_t stream) {
   const int64_t tiles = (rows + kRows - 1) / kRows;
-  if (tiles == 0 || K == 0) return NVFP4_OK;
+  const int64_t n_col = col_amax != nullptr ? static_cast<int64_t>(E) * K : 0;
+  if (n_col == 0 && (tiles == 0 || K == 0)) return NVFP4_OK;
   NVFP4_SPANS(SpanList{}
                   .add(x, static_cast<size_t>(rows) * K * 2, false)
                   .routing(routing)
@@ -238,6 +242,13 @@ nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t rows, in
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return NVFP4_ERR_CUDA;
+  if (n_col > 0) {
+    const int64_t blocks = std::min<int64_t>((n_col + 255) / 256, 2 * static_cast<int64_t>(sms));
+    zero_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(col_amax, n_col);
+    const nvfp4_status z = cuda_status(cudaGetLastError());
+    if (z != NVFP4_OK) return z;
+  }
+  if (tiles == 0 || K == 0) return NVFP4_OK;
   const int cn = amax_cluster(K, tiles, sms);
   const size_t smem = static_cast<size_t>(amax_cta_cols(K, cn)) * sizeof(uint32_t) + sizeof(int32_t) * (E + 1);
   auto kernel = group_amax_kernel<Routing>;
@@ -251,13 +262,17 @@ nvfp4_status launch_amax(const Routing& routing, const void* x, int64_t rows, in
   cfg.blockDim = dim3(kAmaxThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  // programmatic after the zeroing (its reads of x overlap it; its atomics
+  // wait for it); a plain launch when there is no zeroing to overlap
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(cn);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n_col > 0 ? 2 : 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, routing, static_cast<const uint4*>(x),
                                         static_cast<int32_t>(K), static_cast<int32_t>(cn),
                                         row_amax, col_amax));
@@ -561,11 +576,6 @@ nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
   static thread_local HostRouting routing;
   s = host_routing(m_splits_host, num_groups, sum_M, routing);
   if (s != NVFP4_OK) return s;
-  if (col_amax != nullptr && num_groups > 0 && K > 0) {
-    s = cuda_status(cudaMemsetAsync(col_amax, 0, static_cast<size_t>(num_groups) * K * sizeof(float),
-                                    stream));
-    if (s != NVFP4_OK) return s;
-  }
   return launch_amax(routing, x_bf16, sum_M, K, num_groups, row_amax, col_amax, stream);
 }
 
@@ -607,12 +617,6 @@ nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_row
   if (!aligned(row_amax, 4) || !aligned(col_amax, 4)) return NVFP4_ERR_UNSUPPORTED;
   s = cuda_status(cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream));
   if (s != NVFP4_OK) return s;
-  if (col_amax != nullptr && num_groups > 0 && K > 0) {
-    s = cuda_status(cudaMemsetAsync(col_amax, 0, static_cast<size_t>(num_groups) * K * sizeof(float),
-                                    stream));
-    if (s != NVFP4_OK) return s;
-  }
-  if (K == 0) return NVFP4_OK;
   return launch_amax(routing, x_bf16, capacity_rows, K, num_groups, row_amax, col_amax, stream);
 }
 
