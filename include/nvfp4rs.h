@@ -55,9 +55,10 @@
  *    NVFP4_ERR_INVALID_ARG). Else NVFP4_ERR_UNSUPPORTED: every group size
  *    m_g % 16 == 0 (the colwise block height), num_groups <=
  *    NVFP4_MAX_GROUPS, rows < 2^31, and every pointer 16-byte aligned. The
- *    one-launch calls and the 128x4-tiled scale layout also need
+ *    128x4-tiled scale layout and the graph-safe one-launch call also need
  *    K % 128 == 0 and m_g % 128 == 0 (the 128-row alignment of the grouped
- *    GEMM's scale layout); the MXFP4 calls need K % 32 == 0 (else
+ *    GEMM's scale layout; the host-split one-launch calls run other routings
+ *    as two launches); the MXFP4 calls need K % 32 == 0 (else
  *    NVFP4_ERR_INVALID_ARG) and m_g % 32 == 0 (their block size). 128-row tiles inside one group on the
  *    128-row grid, with K % 128 == 0, take the fastest path; the rest is
  *    handled at the tile's edges in the same kernel (a 128-row tile may then
@@ -236,10 +237,14 @@ NVFP4RS_API size_t nvfp4_group_quantize_workspace_bytes(int64_t capacity_rows, i
  *                   workspace must be ordered on one stream. After the call
  *                   word 1 is nonzero only if a bounded wait inside the kernel
  *                   gave up (not expected; the outputs are then incomplete).
- * Every group must be a multiple of 128 rows and K % 128 == 0 (else
- * NVFP4_ERR_UNSUPPORTED); for other shapes use the two calls. With no direction requested
- * nothing is enqueued. Memsets of the workspace header, row_amax and
- * col_amax, then one launch.
+ * The single launch takes routings whose groups are all multiples of 128
+ * rows with K % 128 == 0. Any other routing the two-step calls accept
+ * (groups of multiples of 16 rows, K % 16 == 0) runs here as those two
+ * launches -- the same outputs, the workspace left untouched -- except with
+ * the 128x4-tiled scale layout, which needs 128-row groups and
+ * K % 128 == 0 (else NVFP4_ERR_UNSUPPORTED). With no direction requested
+ * nothing is enqueued. Single launch: memsets of the workspace header,
+ * row_amax and col_amax, then the kernel.
  */
 NVFP4RS_API nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
                                   const int64_t* m_splits_host, int32_t num_groups,
@@ -269,7 +274,8 @@ NVFP4RS_API nvfp4_status nvfp4_group_quantize_graphsafe(const void* x_bf16, int6
 /*
  * nvfp4_group_quantize without a workspace argument: the same one-launch
  * kernel, same arguments and outputs (byte-identical), with its scratch in a
- * static device array inside the library. This call has no counterpart in
+ * static device array inside the library; routings the single launch does
+ * not take run as the two launches, as in nvfp4_group_quantize. This call has no counterpart in
  * the pages the method follows. It is for callers that cannot hand over
  * device memory at the call site: a C caller with no device allocator of
  * its own, or one that must not allocate there (cudaMalloc synchronises the

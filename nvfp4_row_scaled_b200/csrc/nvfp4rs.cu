@@ -562,6 +562,21 @@ nvfp4_status launch_dequant(const uint8_t* data, const uint8_t* scale, const flo
                                         rows, cols, reinterpret_cast<float4*>(out_f32)));
 }
 
+// The host-split one-launch calls on a routing the single-launch kernel does
+// not take (a group not a multiple of 128 rows, or K % 128 != 0): the grouped
+// amax and the grouped cast, the two launches of the two-step calls, with the
+// same outputs. The 128x4-tiled layout needs 128-row groups either way.
+nvfp4_status quantize_two_launches(const HostRouting& routing, const void* x, int64_t rows, int64_t K, int32_t E,
+                                   float* row_amax, float* col_amax, const nvfp4_outputs* out, bool do_row,
+                                   bool do_col, cudaStream_t stream) {
+  if (out->scale_layout == NVFP4_SCALE_TILED_128X4) return NVFP4_ERR_UNSUPPORTED;
+  float* ra = do_row ? row_amax : nullptr;
+  float* ca = do_col ? col_amax : nullptr;
+  const nvfp4_status s = launch_amax(routing, x, rows, K, E, ra, ca, stream);
+  if (s != NVFP4_OK) return s;
+  return launch_cast(routing, x, rows, K, E, ra, ca, out, do_col, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -667,7 +682,7 @@ nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
                                   const int64_t* m_splits_host, int32_t num_groups, float* row_amax,
                                   float* col_amax, const nvfp4_outputs* out, void* workspace,
                                   size_t workspace_bytes, cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups, /*k128=*/true);
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
@@ -676,9 +691,12 @@ nvfp4_status nvfp4_group_quantize(const void* x_bf16, int64_t sum_M, int64_t K,
                      workspace_bytes, 0);
   if (s != NVFP4_OK) return s;
   static thread_local HostRouting routing;
-  s = host_routing(m_splits_host, num_groups, sum_M, routing, kRows);  // one launch: 128-row groups
+  bool all_128 = true;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kBlockRows, &all_128);
   if (s != NVFP4_OK) return s;
   if (!do_row && !do_col) return NVFP4_OK;
+  if (!all_128 || K % kCols != 0) return quantize_two_launches(routing, x_bf16, sum_M, K, num_groups, row_amax,
+                                                               col_amax, out, do_row, do_col, stream);
   // the rows accumulate straight into row_amax
   s = zero_quantize_state(workspace, num_groups, row_amax, sum_M, do_row, col_amax, K, do_col, stream);
   if (s != NVFP4_OK) return s;
@@ -724,7 +742,7 @@ nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int
                                           const int64_t* m_splits_host, int32_t num_groups,
                                           float* row_amax, float* col_amax, const nvfp4_outputs* out,
                                           cudaStream_t stream) {
-  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups, /*k128=*/true);
+  nvfp4_status s = check_shape(x_bf16, sum_M, K, num_groups);
   if (s != NVFP4_OK) return s;
   bool do_row = false, do_col = false;
   s = check_outputs(out, sum_M, K, num_groups, do_row, do_col);
@@ -735,9 +753,12 @@ nvfp4_status nvfp4_group_quantize_noalloc(const void* x_bf16, int64_t sum_M, int
   // the static scratch holds the header of at most NVFP4_MAX_GROUPS groups
   if (quant_ws_header_words(num_groups) > kNoAllocScratchWords) return NVFP4_ERR_UNSUPPORTED;
   static thread_local HostRouting routing;
-  s = host_routing(m_splits_host, num_groups, sum_M, routing, kRows);  // one launch: 128-row groups
+  bool all_128 = true;
+  s = host_routing(m_splits_host, num_groups, sum_M, routing, kBlockRows, &all_128);
   if (s != NVFP4_OK) return s;
   if (!do_row && !do_col) return NVFP4_OK;
+  if (!all_128 || K % kCols != 0) return quantize_two_launches(routing, x_bf16, sum_M, K, num_groups, row_amax,
+                                                               col_amax, out, do_row, do_col, stream);
   uint32_t* scratch = noalloc_scratch();
   if (scratch == nullptr) return NVFP4_ERR_CUDA;
   // zeroed here on `stream`: item counter, abort word, done counters; the

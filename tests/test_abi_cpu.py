@@ -211,18 +211,28 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
 
 
 def test_k_multiple_of_128_only_where_needed(L):
-    """The two-step calls take any K % 16 == 0; the one-launch, MXFP4 and
-    tiled-scale paths need K % 128 == 0 and refuse other K up front."""
+    """The two-step calls take any K % 16 == 0, and so do the host-split
+    one-launch calls (other routings run as the two launches); the
+    graph-safe one-launch call and the tiled-scale layout need K % 128 == 0
+    and refuse other K up front, before anything is enqueued."""
     arr = (ctypes.c_int64 * 1)(256)
     o = abi.Outputs(row_data=0x10000, row_scale=0x10000, row_s2=0x10000,
                     col_data=0x10000, col_scale=0x10000, col_s2=0x10000)
-    ws = abi.nvfp4_group_quantize_workspace_bytes(0, 1)
+    ws = abi.nvfp4_group_quantize_workspace_bytes(256, 1)
+    assert L.nvfp4_group_quantize_graphsafe(FAKE, 256, 144, FAKE, FAKE, 1, FAKE, FAKE, ctypes.byref(o), FAKE,
+                                            ws, FAKE, None) == abi.NVFP4_ERR_UNSUPPORTED
+    o.scale_layout = abi.NVFP4_SCALE_TILED_128X4
     assert L.nvfp4_group_quantize(FAKE, 256, 144, arr, 1, FAKE, FAKE, ctypes.byref(o), FAKE, ws, None) == \
         abi.NVFP4_ERR_UNSUPPORTED
     assert L.nvfp4_group_quantize_noalloc(FAKE, 256, 144, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
         abi.NVFP4_ERR_UNSUPPORTED
-    o.scale_layout = abi.NVFP4_SCALE_TILED_128X4
     assert L.nvfp4_group_cast(FAKE, 256, 144, arr, 1, FAKE, FAKE, ctypes.byref(o), None) == \
         abi.NVFP4_ERR_UNSUPPORTED
     assert L.nvfp4_group_cast_graphsafe(FAKE, 256, 144, FAKE, FAKE, 1, FAKE, FAKE, ctypes.byref(o), FAKE,
                                         None) == abi.NVFP4_ERR_UNSUPPORTED
+    # 128-row groups are needed by the tiled layout in every call
+    arr2 = (ctypes.c_int64 * 2)(48, 208)
+    assert L.nvfp4_group_quantize(FAKE, 256, 128, arr2, 2, FAKE, FAKE, ctypes.byref(o), FAKE, ws, None) == \
+        abi.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_group_cast(FAKE, 256, 128, arr2, 2, FAKE, FAKE, ctypes.byref(o), None) == \
+        abi.NVFP4_ERR_UNSUPPORTED

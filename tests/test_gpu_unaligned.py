@@ -10,8 +10,9 @@ multiple of 16 (the rowwise block width); the last 128-column tile may then
 be partial. Checked byte for byte against the oracle, host-split and
 graph-safe (which must also agree with each other, and leave every byte past
 the routed rows untouched), in both directions and in each alone; uniform
-graph-safe routing (no first_dims / tensor_offsets); the one-launch call,
-which keeps 128-row groups and K % 128 == 0, refuses the rest.
+graph-safe routing (no first_dims / tensor_offsets); the host-split
+one-launch calls, whose single launch keeps 128-row groups and K % 128 == 0,
+run the rest as the two launches.
 """
 import numpy as np
 import pytest
@@ -168,18 +169,69 @@ def test_graphsafe_k_not_multiple_of_128_matches_host_split_and_leaves_tail():
         assert np.all(full[k][c:].view(np.uint8) == SENTINEL), k
 
 
-def test_k_not_multiple_of_128_refused_by_one_launch_and_tiled():
+def test_tiled_layout_refuses_k_not_multiple_of_128():
     K = 144
     splits = [128, 128]
     x = torch.zeros(256, K, dtype=torch.bfloat16, device="cuda")
     ra, ca = abi.alloc_amax(256, K, 2)
     out = abi.alloc_outputs(256, K, 2)
-    with pytest.raises(abi.NVFP4Error) as e:
-        abi.nvfp4_group_quantize(x, splits, ra, ca, out, abi.alloc_workspace(0, 2))
-    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
-    with pytest.raises(abi.NVFP4Error) as e:
-        abi.nvfp4_group_cast(x, splits, ra, ca, out, scale_layout=abi.NVFP4_SCALE_TILED_128X4)
-    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
+    for call in (lambda: abi.nvfp4_group_cast(x, splits, ra, ca, out, scale_layout=abi.NVFP4_SCALE_TILED_128X4),
+                 lambda: abi.nvfp4_group_quantize(x, splits, ra, ca, out, abi.alloc_workspace(0, 2),
+                                                  scale_layout=abi.NVFP4_SCALE_TILED_128X4)):
+        with pytest.raises(abi.NVFP4Error) as e:
+            call()
+        assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
+
+
+ONE_LAUNCH_CASES = [CASES[1], CASES[3], CASES[6], KCASES[0], KCASES[3], KCASES[4]]
+
+
+@pytest.mark.parametrize("K,splits,dist,seed", ONE_LAUNCH_CASES)
+def test_one_launch_calls_take_every_routing(K, splits, dist, seed):
+    """The host-split one-launch calls run a routing their single launch does
+    not take (groups off the 128-row grid, K % 128 != 0) as the two launches:
+    byte-identical to the oracle, workspace untouched."""
+    w = workloads.random_case(seed, K, splits, dist=dist)
+    want = oracle_cast(w.x, splits)
+    xd = w.x.cuda()
+    R, E = xd.shape[0], len(splits)
+    for name in ("workspace", "noalloc"):
+        ra, ca = abi.alloc_amax(R, K, E)
+        out = abi.alloc_outputs(R, K, E)
+        for t in [ra, ca, *out.values()]:
+            t.view(torch.uint8).fill_(SENTINEL)
+        if name == "workspace":
+            ws = abi.alloc_workspace(0, E)
+            ws.fill_(SENTINEL)
+            abi.nvfp4_group_quantize(xd, splits, ra, ca, out, ws)
+        else:
+            abi.nvfp4_group_quantize_noalloc(xd, splits, ra, ca, out)
+        torch.cuda.synchronize()
+        got = {k: v.cpu().numpy() for k, v in out.items()}
+        got["row_amax"], got["col_amax"] = ra.cpu().numpy(), ca.cpu().numpy()
+        assert_identical(got, want, keys=ALL, what=f"{name} K={K} {splits}")
+        if name == "workspace":
+            assert bool((ws == SENTINEL).all()), "the two-launch path leaves the workspace untouched"
+
+
+@pytest.mark.parametrize("rows,cols", [(True, False), (False, True)])
+def test_one_launch_calls_unaligned_single_direction(rows, cols):
+    splits = [48, 0, 208, 16]
+    w = workloads.random_case(87, 400, splits, dist="wide")
+    xd = w.x.cuda()
+    R, K, E = xd.shape[0], xd.shape[1], len(splits)
+    ra, ca = abi.alloc_amax(R, K, E)
+    out = abi.alloc_outputs(R, K, E, row=rows, col=cols)
+    abi.nvfp4_group_quantize(xd, splits, ra if rows else None, ca if cols else None, out,
+                             abi.alloc_workspace(0, E))
+    torch.cuda.synchronize()
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    if rows:
+        got["row_amax"] = ra.cpu().numpy()
+    if cols:
+        got["col_amax"] = ca.cpu().numpy()
+    want = oracle_cast(w.x, splits, rows=rows, cols=cols)
+    assert_identical(got, want, keys=list(want.keys()), what=f"rows={rows} cols={cols}")
 
 
 @pytest.mark.parametrize("E,m", [(4, 128), (10, 48)])
@@ -214,15 +266,14 @@ def test_graphsafe_group_not_multiple_of_16_is_unsupported():
         assert np.all(full[k].view(np.uint8) == SENTINEL), k
 
 
-def test_one_launch_refuses_unaligned_groups():
+def test_graphsafe_one_launch_refuses_unaligned_groups():
+    """The graph-safe one-launch call keeps its single launch and 128-row
+    groups: the device routing check reports the rest."""
     K = 256
     splits = [48, 208]
     x = torch.zeros(sum(splits), K, dtype=torch.bfloat16, device="cuda")
     ra, ca = abi.alloc_amax(sum(splits), K, 2)
     out = abi.alloc_outputs(sum(splits), K, 2)
-    with pytest.raises(abi.NVFP4Error) as e:
-        abi.nvfp4_group_quantize(x, splits, ra, ca, out, abi.alloc_workspace(0, 2))
-    assert e.value.status == abi.NVFP4_ERR_UNSUPPORTED
     fd, offs = abi.routing_tensors(splits, K)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     abi.nvfp4_group_quantize_graphsafe(x, fd, offs, ra, ca, out, abi.alloc_workspace(sum(splits), 2), status)
