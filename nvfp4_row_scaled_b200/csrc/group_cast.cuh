@@ -101,6 +101,10 @@ __device__ __forceinline__ void st_global_u2_hint(void* p, uint2 v, uint64_t pol
   asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y),
                "l"(policy) : "memory");
 }
+__device__ __forceinline__ void st_global_u32_hint(void* p, uint32_t v, uint64_t policy) {
+  if (!NVFP4_STORE_OK(p, 4)) return;
+  asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
+}
 __device__ __forceinline__ void st_global_u4_hint(void* p, uint4 v, uint64_t policy) {
   if (!NVFP4_STORE_OK(p, 16)) return;
   asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
@@ -148,14 +152,15 @@ __device__ __forceinline__ void st_global_u32(uint8_t* p, uint32_t v) {
 
 // The codes of a lane's 16 x 8 patch, once the multipliers are known: renc[i]
 // multiplies row i (rowwise codes, stored straight to rdst + i * row_pitch
-// when row_store), cenc2[q] the column pair (2q, 2q+1) (colwise codes, handed
-// to col_sink(half, cw): cw[q] holds rows 8*half .. 8*half+7 of column q, row
-// 8*half in the low nibble). Shared by the NVFP4 and the MXFP4 casts.
-template <class ColSink>
+// when row_store; with kRowHint under the L2 policy row_policy), cenc2[q] the
+// column pair (2q, 2q+1) (colwise codes, handed to col_sink(half, cw): cw[q]
+// holds rows 8*half .. 8*half+7 of column q, row 8*half in the low nibble).
+// Shared by the NVFP4 and the MXFP4 casts.
+template <bool kRowHint = false, class ColSink>
 __device__ __forceinline__ void encode_codes(const uint4 (&v)[16], const float (&renc)[16],
                                              const uint64_t (&cenc2)[4], bool do_row, bool do_col,
                                              uint8_t* rdst, size_t row_pitch, bool row_store,
-                                             ColSink&& col_sink) {
+                                             ColSink&& col_sink, uint64_t row_policy = 0) {
 #pragma unroll
   for (int half = 0; half < 2; half++) {
     uint32_t A[4], B[4];  // per row pair: codes of columns 0..3 / 4..7
@@ -170,8 +175,13 @@ __device__ __forceinline__ void encode_codes(const uint4 (&v)[16], const float (
         const uint32_t w0 = e2m1_pairs(mul2x(x0[0], e0), mul2x(x0[1], e0), mul2x(x0[2], e0), mul2x(x0[3], e0));
         const uint32_t w1 = e2m1_pairs(mul2x(x1[0], e1), mul2x(x1[1], e1), mul2x(x1[2], e1), mul2x(x1[3], e1));
         if (row_store) {  // false for a 16-row block past the routed rows
-          st_global_u32(rdst + i * row_pitch, w0);
-          st_global_u32(rdst + (i + 1) * row_pitch, w1);
+          if (kRowHint) {
+            st_global_u32_hint(rdst + i * row_pitch, w0, row_policy);
+            st_global_u32_hint(rdst + (i + 1) * row_pitch, w1, row_policy);
+          } else {
+            st_global_u32(rdst + i * row_pitch, w0);
+            st_global_u32(rdst + (i + 1) * row_pitch, w1);
+          }
         }
       }
       if (do_col) {
@@ -231,11 +241,11 @@ __device__ __forceinline__ void col_senc_pairs(const float* col_senc, int cc, ui
 // cc ^ 1 (the neighbouring lane). cse: S_enc of the lane's 8 columns in
 // pairs (2q, 2q+1). kExact selects the IEEE-divide block scales (tiles with a
 // row or column amax outside the shortcut's range).
-template <bool kExact, class ColSink>
+template <bool kExact, bool kRowHint = false, class ColSink>
 __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeTables& tab, const uint64_t (&cse)[4],
                                              uint8_t* col_stg, uint8_t* row_stg, bool do_row, bool do_col, int cc,
                                              int rb, uint8_t* rdst, size_t row_pitch, bool row_store,
-                                             ColSink&& col_sink) {
+                                             ColSink&& col_sink, uint64_t row_policy = 0) {
   const int rl = 16 * rb;
   const bool odd = cc & 1;
 
@@ -305,7 +315,7 @@ __device__ __forceinline__ void encode_patch(const uint4 (&v)[16], const EncodeT
   }
 
   // -------------------------------------------------------------- codes
-  encode_codes(v, renc, cenc2, do_row, do_col, rdst, row_pitch, row_store, col_sink);
+  encode_codes<kRowHint>(v, renc, cenc2, do_row, do_col, rdst, row_pitch, row_store, col_sink, row_policy);
 }
 
 // The 128x4-tiled scale layout (the grouped GEMM's swizzle contract; see the

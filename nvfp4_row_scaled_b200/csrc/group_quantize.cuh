@@ -428,7 +428,11 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
   const int rb = 4 * (w >> 1) + hb;  // 16-row block of the tile, 0..7
   const int rl = 16 * rb;
   const size_t row_pitch = static_cast<size_t>(K) >> 1;
-  const uint64_t keep = policy_evict_last();
+  // every output of a cast item (codes and scales) is stored evict-first, so
+  // that the tiles still waiting in L2 for their cast item keep their place
+  // (measured against the default policy for rowwise codes and evict-last
+  // scales: 1.61 instead of 1.69 GB read from DRAM at the DeepSeek-V3 shape,
+  // 0.517 instead of 0.524 ms; 1024 tokens: 211 instead of 221 us)
   const uint64_t once = policy_evict_first();
   const int bar_id = 1 + j;
 
@@ -481,7 +485,7 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
       const int tp = item_tile(prev_item), rtp = tp / n_ct;
       store_scales<kTiled>(pg.col_scale[(k - 1) & 1], pg.row_scale[(k - 1) & 1], out, K, rs.off[prev_g],
                            rs.off[prev_g + 1] - rs.off[prev_g], rtp * kRows, (tp - rtp * n_ct) * kCols, gt,
-                           do_row, do_col, keep);
+                           do_row, do_col, once);
     }
     if (item < 0) break;  // the end mark
     prev_item = item;
@@ -500,11 +504,11 @@ group_quantize_kernel(const __grid_constant__ Routing routing, const __grid_cons
       uint64_t cse[4];
       if (do_col) col_senc_pairs(pg.col_senc[s], cc, cse);
       if (any_slow)
-        encode_patch<true>(v, tab, cse, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
-                           row_pitch, true, sink);
+        encode_patch<true, true>(v, tab, cse, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb,
+                                 rdst, row_pitch, true, sink, once);
       else
-        encode_patch<false>(v, tab, cse, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb, rdst,
-                            row_pitch, true, sink);
+        encode_patch<false, true>(v, tab, cse, pg.col_scale[k & 1], pg.row_scale[k & 1], do_row, do_col, cc, rb,
+                                  rdst, row_pitch, true, sink, once);
     } else {
       // ------------------------------------------------------------ A item
       // column maxima over the warp's 64 rows (lanes hb = 0..3 share the
