@@ -104,3 +104,31 @@ def test_dequantize_matches_oracle_both_directions():
         abi.nvfp4_dequantize(d, s, s2, K, m, xh)
         want = oracle.dequantize(d.cpu().numpy(), s.cpu().numpy(), s2.cpu().numpy(), K, m)
         assert_identical({"x": xh.cpu().numpy()}, {"x": want}, what=f"colwise dequant g={g}")
+
+
+@pytest.mark.parametrize("K,splits", [(7168, [256, 0, 384, 128]), (2048, [48, 208, 16, 0, 112]), (144, [128, 32])])
+def test_amax_waits_for_its_zeroing(K, splits):
+    """col_amax starts as all-ones words (larger, as unsigned, than any float
+    the atomic max can bring): the amax call's zeroing kernel must finish
+    before the first atomic of the amax kernel launched programmatically
+    after it, on every call (TransformerEngine #3649, Description: the amax
+    step's column amax vector is the per-group maximum)."""
+    w = workloads.random_case(91, K, splits, dist="wide")
+    want = oracle_cast(w.x, splits)
+    xd = w.x.cuda()
+    R, E = xd.shape[0], len(splits)
+    ra, ca = abi.alloc_amax(R, K, E)
+    for call in range(3):
+        ca.view(torch.int32).fill_(-1)
+        ra.view(torch.int32).fill_(-1)
+        abi.nvfp4_group_amax(xd, splits, ra, ca)
+        torch.cuda.synchronize()
+        assert_identical({"row_amax": ra.cpu().numpy(), "col_amax": ca.cpu().numpy()}, want,
+                         keys=["row_amax", "col_amax"], what=f"call {call}")
+    fd, offs = abi.routing_tensors(splits, K)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ca.view(torch.int32).fill_(-1)
+    abi.nvfp4_group_amax_graphsafe(xd, fd, offs, ra, ca, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert_identical({"col_amax": ca.cpu().numpy()}, want, keys=["col_amax"], what="graph-safe")
