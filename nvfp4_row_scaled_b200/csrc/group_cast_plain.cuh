@@ -46,9 +46,13 @@
 //    (store_scales_general).
 // Ring invariants (tile k of a group): the stage completes phase k % 2 of
 // its mbarrier, amax slot k % 3, tile info entry k % 4, scale staging k % 2.
-// The refill issued after tile k's barrier writes the stage, slot (k+1) % 3
-// and entry (k+1) % 4; every read of those by tiles k and k-1 that is not
-// already done happens after that barrier and touches other entries.
+// After tile k's barrier one thread loads tile k+1 into the stage and slot
+// (k+1) % 3 (its info, entry (k+1) % 4, was written after tile k-1's
+// barrier) and writes tile k+2's info into entry (k+2) % 4. Every read of
+// the stage by tile k happened before that barrier; what tile k reads after
+// it (slot k % 3, entry k % 4) and tile k-1's scale stores (entry
+// (k-1) % 4, staging (k-1) % 2) are other entries; entry (k+2) % 4 was last
+// read by tile k-2, before tile k-1's barrier.
 #pragma once
 
 #include "group_cast.cuh"
