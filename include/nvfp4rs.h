@@ -138,7 +138,9 @@ typedef struct {
  *   row_amax       device fp32 [sum_M], or NULL to skip rows
  *   col_amax       device fp32 [num_groups*K], or NULL to skip columns; it is
  *                  zeroed on `stream` by this call first
- * One launch (plus one memset of col_amax).
+ * Two launches when col_amax is given: a kernel that zeroes col_amax, then the
+ * amax kernel, launched programmatically so that its reads of x overlap the
+ * zeroing (its atomics on col_amax wait for it); else the amax kernel alone.
  */
 NVFP4RS_API nvfp4_status nvfp4_group_amax(const void* x_bf16, int64_t sum_M, int64_t K,
                               const int64_t* m_splits_host, int32_t num_groups,
@@ -184,7 +186,7 @@ NVFP4RS_API nvfp4_status nvfp4_group_cast(const void* x_bf16, int64_t sum_M, int
  * Uniform groups: with first_dims_dev and tensor_offsets_dev both NULL every
  * group has capacity_rows / num_groups rows (which must divide exactly, else
  * NVFP4_ERR_INVALID_ARG; a multiple of 16, else NVFP4_ERR_UNSUPPORTED).
- * One launch plus memsets of status and col_amax.
+ * A memset of status, then the launches of nvfp4_group_amax.
  */
 NVFP4RS_API nvfp4_status nvfp4_group_amax_graphsafe(const void* x_bf16, int64_t capacity_rows, int64_t K,
                                         const int64_t* first_dims_dev,
