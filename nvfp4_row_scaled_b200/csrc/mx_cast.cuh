@@ -129,7 +129,9 @@ constexpr size_t mx_smem_bytes(int E) {
 }
 
 // One thread of the group: tile (rt, ct) -- the group's k-th -- into the
-// stage with its tile info (as plain_issue, without amax copies).
+// stage with its tile info (as plain_info and plain_load of the NVFP4 cast
+// together, without amax copies; the info is written when the tile is issued,
+// one tile ahead, and read after the next barrier).
 __device__ __forceinline__ void mx_issue(MxGroup& pg, uint8_t* stage, const CUtensorMap* map, int k, int rt,
                                          int ct, const RoutingSmem& rs, int K, bool k128) {
   const int32_t r0 = rt * kRows;
